@@ -1,0 +1,246 @@
+"""Gated delta rule (KDA / Gated DeltaNet) on B200: Python binding.
+
+A thin ctypes layer over the C ABI in ``include/gated_delta.h``
+(``libgated_delta.so``, built in-tree for sm_100a).  It only marshals
+arguments: every step of the computation runs in the library's CUDA kernels.
+PyTorch is used for device memory and streams.  There is no CPU path: if the
+library is missing or no CUDA device is present the calls raise.
+
+Operator (thethings.ai "The argument, in one page", table "Everything, in
+one table", rows "KDA" and "Gated DeltaNet"; column-vector keys):
+
+    S_t = Diag(exp(g_t)) (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+    o_t = S_t^T q_t
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import threading
+from typing import Optional, Tuple
+
+__all__ = [
+    "lib", "library_path", "KdaError", "kda_chunk_fwd", "gdn_chunk_fwd", "kda_decode_step",
+    "gdn_decode_step", "chunk_workspace_size", "check_device_status", "EXPORTED_SYMBOLS",
+    "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
+    "KDA_ERR_DEVICE_CHECK", "KDA_ERR_WORKSPACE",
+]
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+library_path = os.path.join(_PKG, "libgated_delta.so")
+
+KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_DEVICE_CHECK, \
+    KDA_ERR_WORKSPACE = range(6)
+KDA_F32, KDA_BF16 = 0, 1
+
+EXPORTED_SYMBOLS = (
+    "kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "gdn_chunk_fwd",
+    "gdn_chunk_fwd_workspace_size", "kda_decode_step", "gdn_decode_step",
+    "kda_check_device_status", "kda_status_string", "kda_last_error", "kda_abi_version",
+)
+
+_lock = threading.Lock()
+_lib = None
+
+_vp, _fp, _i32, _sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+_SIGS = {
+    "kda_chunk_fwd": ([_vp] * 9 + [_i32] * 6 + [ctypes.c_int, _vp, _sz, _vp], ctypes.c_int),
+    "gdn_chunk_fwd": ([_vp] * 9 + [_i32] * 7 + [ctypes.c_int, _vp, _sz, _vp], ctypes.c_int),
+    "kda_chunk_fwd_workspace_size": ([_i32] * 6 + [ctypes.c_int], _sz),
+    "gdn_chunk_fwd_workspace_size": ([_i32] * 7 + [ctypes.c_int], _sz),
+    "kda_decode_step": ([_vp] * 7 + [_i32] * 4 + [ctypes.c_int, _vp], ctypes.c_int),
+    "gdn_decode_step": ([_vp] * 7 + [_i32] * 5 + [ctypes.c_int, _vp], ctypes.c_int),
+    "kda_check_device_status": ([_vp, _vp, ctypes.POINTER(_i32)], ctypes.c_int),
+    "kda_status_string": ([ctypes.c_int], ctypes.c_char_p),
+    "kda_last_error": ([], ctypes.c_char_p),
+    "kda_abi_version": ([], _i32),
+}
+
+
+class KdaError(RuntimeError):
+    def __init__(self, status: int, detail: str):
+        self.status = status
+        super().__init__(f"{detail} (status {status})")
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libgated_delta.so`` (raises if it has not been built)."""
+    global _lib
+    with _lock:
+        if _lib is None:
+            if not os.path.exists(library_path):
+                raise ImportError(
+                    f"{library_path} is missing: build it with "
+                    "`python -m gated_delta_rule_87_b200.build` (nvcc, sm_100a)")
+            L = ctypes.CDLL(library_path)
+            for name, (args, res) in _SIGS.items():
+                f = getattr(L, name)
+                f.argtypes = args
+                f.restype = res
+            _lib = L
+    return _lib
+
+
+def _check(status: int, what: str):
+    if status != KDA_OK:
+        L = lib()
+        msg = L.kda_last_error().decode() or L.kda_status_string(status).decode()
+        raise KdaError(status, f"{what}: {msg}")
+
+
+# --------------------------------------------------------------------------- #
+# torch plumbing
+# --------------------------------------------------------------------------- #
+def _torch():
+    import torch
+    return torch
+
+
+def _dtype_code(t) -> int:
+    torch = _torch()
+    if t.dtype == torch.bfloat16:
+        return KDA_BF16
+    if t.dtype == torch.float32:
+        return KDA_F32
+    raise TypeError(f"q/k/v must be bfloat16 or float32, got {t.dtype}")
+
+
+def _ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _stream_handle(stream, device) -> int:
+    torch = _torch()
+    s = stream if stream is not None else torch.cuda.current_stream(device)
+    return s.cuda_stream
+
+
+def _f32(t, name):
+    torch = _torch()
+    if t is not None and t.dtype != torch.float32:
+        raise TypeError(f"{name} must be float32")
+    return t
+
+
+def chunk_workspace_size(B: int, T: int, H_qk: int, H_v: int, d_k: int, d_v: int,
+                         num_seqs: int, io_dtype: int, gate: str = "channel") -> int:
+    L = lib()
+    if gate == "channel":
+        return int(L.kda_chunk_fwd_workspace_size(B, T, H_v, d_k, d_v, num_seqs, io_dtype))
+    return int(L.gdn_chunk_fwd_workspace_size(B, T, H_qk, H_v, d_k, d_v, num_seqs, io_dtype))
+
+
+def _alloc_workspace(nbytes: int, device):
+    torch = _torch()
+    # 256-byte alignment: torch's caching allocator returns 512-byte aligned blocks
+    return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
+
+
+def _chunk_fwd(gate, q, k, v, g, beta, initial_state, cu_seqlens, output_final_state,
+               o, final_state, workspace, stream):
+    torch = _torch()
+    if q.dim() != 4:
+        raise ValueError("q, k, v must be [B, T, H, d]")
+    B, T, H_qk, d_k = q.shape
+    H_v, d_v = v.shape[2], v.shape[3]
+    io = _dtype_code(q)
+    if k.dtype != q.dtype or v.dtype != q.dtype:
+        raise TypeError("q, k, v must share a dtype")
+    _f32(g, "g"), _f32(beta, "beta"), _f32(initial_state, "initial_state")
+    if cu_seqlens is not None:
+        if cu_seqlens.dtype != torch.int32:
+            raise TypeError("cu_seqlens must be int32")
+        N = cu_seqlens.numel() - 1
+    else:
+        N = B
+    dev = q.device
+    if o is None:
+        o = torch.empty((B, T, H_v, d_v), dtype=q.dtype, device=dev)
+    if final_state is None and output_final_state:
+        final_state = torch.empty((N, H_v, d_k, d_v), dtype=torch.float32, device=dev)
+    need = chunk_workspace_size(B, T, H_qk, H_v, d_k, d_v, N if cu_seqlens is not None else 0,
+                                io, gate)
+    if workspace is None or workspace.numel() < need:
+        workspace = _alloc_workspace(need, dev)
+    L = lib()
+    args_common = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(o), _ptr(initial_state),
+                   _ptr(final_state), _ptr(cu_seqlens), N]
+    sh = _stream_handle(stream, dev)
+    if gate == "channel":
+        st = L.kda_chunk_fwd(*args_common, B, T, H_v, d_k, d_v, io, _ptr(workspace),
+                             workspace.numel(), sh)
+        _check(st, "kda_chunk_fwd")
+    else:
+        st = L.gdn_chunk_fwd(*args_common, B, T, H_qk, H_v, d_k, d_v, io, _ptr(workspace),
+                             workspace.numel(), sh)
+        _check(st, "gdn_chunk_fwd")
+    return o, final_state, workspace
+
+
+def kda_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *,
+                  output_final_state: bool = True, o=None, final_state=None, workspace=None,
+                  stream=None):
+    """KDA prefill.  q, k [B,T,H,d_k]; v [B,T,H,d_v] (bf16 or fp32); g [B,T,H,d_k]
+    fp32 log-decay; beta [B,T,H] fp32; initial_state [N,H,d_k,d_v] fp32 or None;
+    cu_seqlens int32 [N+1] (device) for packed sequences with B = 1.
+    Returns (o, final_state, workspace)."""
+    return _chunk_fwd("channel", q, k, v, g, beta, initial_state, cu_seqlens,
+                      output_final_state, o, final_state, workspace, stream)
+
+
+def gdn_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *,
+                  output_final_state: bool = True, o=None, final_state=None, workspace=None,
+                  stream=None):
+    """Gated DeltaNet prefill.  q, k [B,T,H_qk,d_k]; v [B,T,H_v,d_v]; g, beta
+    [B,T,H_v] fp32 (scalar log-decay per head-token).  Returns (o, final_state,
+    workspace)."""
+    return _chunk_fwd("scalar", q, k, v, g, beta, initial_state, cu_seqlens,
+                      output_final_state, o, final_state, workspace, stream)
+
+
+def _decode(gate, q, k, v, g, beta, state, o, stream):
+    torch = _torch()
+    N, H_qk, d_k = q.shape
+    H_v, d_v = v.shape[1], v.shape[2]
+    io = _dtype_code(q)
+    _f32(g, "g"), _f32(beta, "beta"), _f32(state, "state")
+    if o is None:
+        o = torch.empty((N, H_v, d_v), dtype=q.dtype, device=q.device)
+    L = lib()
+    sh = _stream_handle(stream, q.device)
+    ptrs = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(o), _ptr(state)]
+    if gate == "channel":
+        _check(L.kda_decode_step(*ptrs, N, H_v, d_k, d_v, io, sh), "kda_decode_step")
+    else:
+        _check(L.gdn_decode_step(*ptrs, N, H_qk, H_v, d_k, d_v, io, sh), "gdn_decode_step")
+    return o
+
+
+def kda_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
+    """One KDA decode step; ``state`` [N,H,d_k,d_v] fp32 is updated in place.
+    q, k [N,H,d_k]; v [N,H,d_v]; g [N,H,d_k]; beta [N,H].  Returns o [N,H,d_v]."""
+    return _decode("channel", q, k, v, g, beta, state, o, stream)
+
+
+def gdn_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
+    """One Gated DeltaNet decode step (scalar gate, q/k heads shared by groups of
+    v heads); ``state`` is updated in place.  Returns o [N,H_v,d_v]."""
+    return _decode("scalar", q, k, v, g, beta, state, o, stream)
+
+
+def check_device_status(workspace, stream=None) -> Tuple[int, int]:
+    """Synchronise ``stream`` and read the device status word of a prefill
+    workspace.  Returns (status, device_code); raises on KDA_ERR_CUDA."""
+    L = lib()
+    code = ctypes.c_int32(0)
+    st = L.kda_check_device_status(_ptr(workspace), _stream_handle(stream, workspace.device),
+                                   ctypes.byref(code))
+    if st == KDA_ERR_CUDA:
+        _check(st, "kda_check_device_status")
+    return st, code.value

@@ -1,0 +1,252 @@
+// C ABI of the gated delta-rule library: argument validation, workspace
+// sizing and dispatch to the kernels.  See include/gated_delta.h.
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <string>
+
+#include "common.cuh"
+#include "gated_delta.h"
+#include "internal.h"
+
+namespace {
+
+thread_local std::string g_last_error;
+
+kda_status_t fail(kda_status_t st, const char *fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return st;
+}
+
+kda_status_t cuda_fail(cudaError_t e, const char *where) {
+  return fail(KDA_ERR_CUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool head_dim_ok(int d) { return d == 64 || d == 128; }
+
+constexpr size_t kStatusBytes = 256;
+
+
+// Validation shared by both prefill entry points.
+kda_status_t check_prefill(const gdr::PrefillArgs &a) {
+  if (!a.q || !a.k || !a.v || !a.g || !a.beta || !a.o)
+    return fail(KDA_ERR_INVALID_ARG, "q, k, v, g, beta and o must be non-NULL");
+  if (a.B <= 0 || a.T < 0 || a.H_qk <= 0 || a.H_v <= 0)
+    return fail(KDA_ERR_INVALID_ARG, "need B > 0, T >= 0, H > 0 (B=%d T=%d H_qk=%d H_v=%d)", a.B,
+                a.T, a.H_qk, a.H_v);
+  if (a.H_v % a.H_qk != 0)
+    return fail(KDA_ERR_INVALID_ARG, "H_v (%d) must be a multiple of H_qk (%d)", a.H_v, a.H_qk);
+  if (!head_dim_ok(a.d_k) || !head_dim_ok(a.d_v))
+    return fail(KDA_ERR_UNSUPPORTED, "d_k and d_v must be 64 or 128 (got %d, %d)", a.d_k, a.d_v);
+  const void *ptrs[] = {a.q, a.k, a.v, a.g, a.beta, a.o, a.initial_state, a.final_state,
+                        a.cu_seqlens};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", p);
+  if (a.cu_seqlens) {
+    if (a.B != 1) return fail(KDA_ERR_INVALID_ARG, "packed sequences (cu_seqlens) need B == 1");
+    if (a.num_seqs < 0) return fail(KDA_ERR_INVALID_ARG, "num_seqs must be >= 0");
+  }
+  if ((int64_t)a.B * a.T > INT32_MAX)
+    return fail(KDA_ERR_INVALID_ARG, "B*T must fit in int32");
+  if (a.o == a.q || a.o == a.k || a.o == a.v)
+    return fail(KDA_ERR_INVALID_ARG, "o must not alias q, k or v");
+  if (!a.workspace) return fail(KDA_ERR_WORKSPACE, "workspace is NULL");
+  if (reinterpret_cast<uintptr_t>(a.workspace) & 255u)
+    return fail(KDA_ERR_WORKSPACE, "workspace must be 256-byte aligned");
+  const size_t need = gdr::prefill_workspace_bytes(a.B * a.T, a.H_v, a.d_k, a.d_v, a.num_seqs, a.bf16);
+  if (a.workspace_bytes < need)
+    return fail(KDA_ERR_WORKSPACE, "workspace has %zu bytes, %zu needed", a.workspace_bytes, need);
+  return KDA_OK;
+}
+
+bool use_tensor_core_path(const gdr::PrefillArgs &a) {
+  return a.bf16 && a.d_k == 128 && a.d_v == 128;
+}
+
+kda_status_t run_prefill(gdr::PrefillArgs &a, cudaStream_t s) {
+  kda_status_t st = check_prefill(a);
+  if (st != KDA_OK) return st;
+  int32_t *status = reinterpret_cast<int32_t *>(a.workspace);
+  cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  if (a.cu_seqlens) {
+    e = gdr::launch_check_cu_seqlens(a.cu_seqlens, a.num_seqs, a.T, status, s);
+    if (e != cudaSuccess) return cuda_fail(e, "cu_seqlens check launch");
+  } else {
+    a.num_seqs = a.B;
+  }
+  if (a.num_seqs == 0 || a.T == 0) {
+    // nothing to compute; final state = initial state
+    if (a.final_state) {
+      const size_t bytes = (size_t)a.num_seqs * a.H_v * a.d_k * a.d_v * sizeof(float);
+      if (bytes) {
+        e = a.initial_state ? cudaMemcpyAsync(a.final_state, a.initial_state, bytes,
+                                              cudaMemcpyDeviceToDevice, s)
+                            : cudaMemsetAsync(a.final_state, 0, bytes, s);
+        if (e != cudaSuccess) return cuda_fail(e, "final state copy");
+      }
+    }
+    return KDA_OK;
+  }
+  a.max_chunks = (int64_t)(a.B * (int64_t)a.T) / gdr::kChunk + a.num_seqs;
+  e = use_tensor_core_path(a) ? gdr::launch_prefill_tc(a, s) : gdr::launch_prefill_f32(a, s);
+  if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
+  return KDA_OK;
+}
+
+}  // namespace
+
+namespace gdr {
+
+__global__ void check_cu_seqlens_kernel(const int32_t *__restrict__ cu, int num_seqs, int T,
+                                        int32_t *status) {
+  bool bad = false;
+  for (int i = threadIdx.x; i <= num_seqs; i += blockDim.x) {
+    const int32_t x = cu[i];
+    if (i == 0 && x != 0) bad = true;
+    if (i == num_seqs && x != T) bad = true;
+    if (i < num_seqs && cu[i + 1] < x) bad = true;
+  }
+  if (__syncthreads_or(bad) && threadIdx.x == 0) *status = KDA_DEVICE_BAD_CU_SEQLENS;
+}
+
+cudaError_t launch_check_cu_seqlens(const int32_t *cu, int num_seqs, int T, int32_t *status,
+                                    cudaStream_t stream) {
+  check_cu_seqlens_kernel<<<1, 256, 0, stream>>>(cu, num_seqs, T, status);
+  return cudaGetLastError();
+}
+
+}  // namespace gdr
+
+extern "C" {
+
+int32_t kda_abi_version(void) { return KDA_ABI_VERSION; }
+
+const char *kda_status_string(kda_status_t s) {
+  switch (s) {
+    case KDA_OK: return "ok";
+    case KDA_ERR_INVALID_ARG: return "invalid argument";
+    case KDA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case KDA_ERR_CUDA: return "CUDA error";
+    case KDA_ERR_DEVICE_CHECK: return "device-side check failed";
+    case KDA_ERR_WORKSPACE: return "workspace missing or too small";
+  }
+  return "unknown status";
+}
+
+const char *kda_last_error(void) { return g_last_error.c_str(); }
+
+size_t kda_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                    int32_t num_seqs, kda_dtype_t io_dtype) {
+  const int n = num_seqs > 0 ? num_seqs : B;
+  return gdr::prefill_workspace_bytes(B * T, H, d_k, d_v, n, io_dtype == KDA_BF16);
+}
+
+size_t gdn_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H_qk, int32_t H_v, int32_t d_k,
+                                    int32_t d_v, int32_t num_seqs, kda_dtype_t io_dtype) {
+  (void)H_qk;
+  const int n = num_seqs > 0 ? num_seqs : B;
+  return gdr::prefill_workspace_bytes(B * T, H_v, d_k, d_v, n, io_dtype == KDA_BF16);
+}
+
+kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, void *o, const float *initial_state,
+                           float *final_state, const int32_t *cu_seqlens, int32_t num_seqs,
+                           int32_t B, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                           kda_dtype_t io_dtype, void *workspace, size_t workspace_bytes,
+                           void *stream) {
+  if (io_dtype != KDA_F32 && io_dtype != KDA_BF16)
+    return fail(KDA_ERR_INVALID_ARG, "io_dtype must be KDA_F32 or KDA_BF16");
+  gdr::PrefillArgs a{};
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = o;
+  a.initial_state = initial_state; a.final_state = final_state;
+  a.cu_seqlens = cu_seqlens; a.num_seqs = cu_seqlens ? num_seqs : B;
+  a.B = B; a.T = T; a.H_qk = H; a.H_v = H; a.d_k = d_k; a.d_v = d_v;
+  a.channel_gate = true; a.bf16 = (io_dtype == KDA_BF16);
+  a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+  return run_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+kda_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, void *o, const float *initial_state,
+                           float *final_state, const int32_t *cu_seqlens, int32_t num_seqs,
+                           int32_t B, int32_t T, int32_t H_qk, int32_t H_v, int32_t d_k,
+                           int32_t d_v, kda_dtype_t io_dtype, void *workspace,
+                           size_t workspace_bytes, void *stream) {
+  if (io_dtype != KDA_F32 && io_dtype != KDA_BF16)
+    return fail(KDA_ERR_INVALID_ARG, "io_dtype must be KDA_F32 or KDA_BF16");
+  gdr::PrefillArgs a{};
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = o;
+  a.initial_state = initial_state; a.final_state = final_state;
+  a.cu_seqlens = cu_seqlens; a.num_seqs = cu_seqlens ? num_seqs : B;
+  a.B = B; a.T = T; a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v;
+  a.channel_gate = false; a.bf16 = (io_dtype == KDA_BF16);
+  a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+  return run_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
+static kda_status_t decode_common(gdr::DecodeArgs &a, kda_dtype_t io_dtype, void *stream) {
+  if (io_dtype != KDA_F32 && io_dtype != KDA_BF16)
+    return fail(KDA_ERR_INVALID_ARG, "io_dtype must be KDA_F32 or KDA_BF16");
+  a.bf16 = (io_dtype == KDA_BF16);
+  if (!a.q || !a.k || !a.v || !a.g || !a.beta || !a.o || !a.state)
+    return fail(KDA_ERR_INVALID_ARG, "q, k, v, g, beta, o and state must be non-NULL");
+  if (a.N < 0 || a.H_qk <= 0 || a.H_v <= 0)
+    return fail(KDA_ERR_INVALID_ARG, "need N >= 0 and H > 0");
+  if (a.H_v % a.H_qk != 0)
+    return fail(KDA_ERR_INVALID_ARG, "H_v (%d) must be a multiple of H_qk (%d)", a.H_v, a.H_qk);
+  if (!head_dim_ok(a.d_k) || !head_dim_ok(a.d_v))
+    return fail(KDA_ERR_UNSUPPORTED, "d_k and d_v must be 64 or 128 (got %d, %d)", a.d_k, a.d_v);
+  if ((int64_t)a.N * a.H_v > INT32_MAX)
+    return fail(KDA_ERR_INVALID_ARG, "N*H must fit in int32");
+  const void *ptrs[] = {a.q, a.k, a.v, a.g, a.beta, a.o, a.state};
+  for (const void *p : ptrs)
+    if (!aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", p);
+  if (a.o == a.q || a.o == a.k || a.o == a.v || a.o == a.state)
+    return fail(KDA_ERR_INVALID_ARG, "o must not alias an input or the state");
+  cudaError_t e = gdr::launch_decode_step(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  return KDA_OK;
+}
+
+kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, void *o, float *state, int32_t N, int32_t H,
+                             int32_t d_k, int32_t d_v, kda_dtype_t io_dtype, void *stream) {
+  gdr::DecodeArgs a{};
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = o; a.state = state;
+  a.N = N; a.H_qk = H; a.H_v = H; a.d_k = d_k; a.d_v = d_v; a.channel_gate = true;
+  return decode_common(a, io_dtype, stream);
+}
+
+kda_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, void *o, float *state, int32_t N, int32_t H_qk,
+                             int32_t H_v, int32_t d_k, int32_t d_v, kda_dtype_t io_dtype,
+                             void *stream) {
+  gdr::DecodeArgs a{};
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = o; a.state = state;
+  a.N = N; a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v; a.channel_gate = false;
+  return decode_common(a, io_dtype, stream);
+}
+
+kda_status_t kda_check_device_status(const void *workspace, void *stream, int32_t *device_code) {
+  if (!workspace) return fail(KDA_ERR_INVALID_ARG, "workspace is NULL");
+  int32_t code = 0;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemcpyAsync(&code, workspace, sizeof(code), cudaMemcpyDeviceToHost, s);
+  if (e == cudaSuccess) e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "reading the device status");
+  if (device_code) *device_code = code;
+  if (code != KDA_DEVICE_OK)
+    return fail(KDA_ERR_DEVICE_CHECK, "device check failed with code %d", code);
+  return KDA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,54 @@
+// Internal launch interfaces between the C ABI layer (api.cu) and the kernels.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stddef.h>
+#include <stdint.h>
+
+namespace gdr {
+
+struct DecodeArgs {
+  const void *q, *k, *v;
+  const float *g, *beta;
+  void *o;
+  float *state;
+  int N, H_qk, H_v, d_k, d_v;
+  bool channel_gate;  // KDA (per-channel) or Gated DeltaNet (scalar)
+  bool bf16;          // io dtype
+};
+
+cudaError_t launch_decode_step(const DecodeArgs &a, cudaStream_t stream);
+
+// Chunk length of the prefill kernels (tokens per chunk).
+constexpr int kChunk = 64;
+
+struct PrefillArgs {
+  const void *q, *k, *v;
+  const float *g, *beta;
+  void *o;
+  const float *initial_state;
+  float *final_state;
+  const int32_t *cu_seqlens;  // device, or nullptr (dense)
+  int num_seqs;               // N
+  int B, T, H_qk, H_v, d_k, d_v;
+  bool channel_gate;
+  bool bf16;
+  // workspace (device); status word at offset 0
+  void *workspace;
+  size_t workspace_bytes;
+  // chunks: an upper bound on the total number of chunks over all sequences
+  int64_t max_chunks;
+};
+
+// Bytes of workspace a prefill call needs (includes the 256-byte status block).
+size_t prefill_workspace_bytes(int T, int H_v, int d_k, int d_v, int num_seqs, bool bf16);
+
+cudaError_t launch_prefill_f32(const PrefillArgs &a, cudaStream_t stream);
+cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream);
+
+// Device-side check of cu_seqlens; writes KDA_DEVICE_BAD_CU_SEQLENS into the
+// status word on failure (kernels then skip all work).
+cudaError_t launch_check_cu_seqlens(const int32_t *cu, int num_seqs, int T, int32_t *status,
+                                    cudaStream_t stream);
+
+}  // namespace gdr

@@ -7,10 +7,13 @@ oracle.  Shapes and distributions follow the workloads stated for the method
 batched decode, long Gated DeltaNet prefill with shared q/k heads, and a
 small all-fp32 Gated DeltaNet case).
 
-Generation recipe (one ``numpy.random.default_rng(seed)`` stream per
-workload, draws in this fixed order):
-
-    [varlen lengths] -> q -> k -> v -> gate -> beta -> initial state
+Generation recipe.  Varlen lengths come first, from
+``numpy.random.default_rng(seed).integers(lo, hi, n, endpoint=True)``.  Every
+tensor is then drawn as standard normals in fp64, in blocks of whole rows along
+its leading axis (about 2^22 elements per block); block b of tensor number
+``tag`` (q = 1, k = 2, v = 3, gate = 4, beta = 5, initial state = 6) comes
+from its own stream ``numpy.random.default_rng([seed, tag, b])``, so blocks
+are drawn in parallel and the result does not depend on the thread count.
 
 * q, k: standard normal in fp64, L2-normalised per (token, head) over d_k in
   fp64, then rounded to the io dtype (round to nearest even for bf16).
@@ -161,12 +164,48 @@ class DecodeInputs:
 # --------------------------------------------------------------------------- #
 # generation
 # --------------------------------------------------------------------------- #
-def _normal(rng, shape) -> np.ndarray:
-    return rng.standard_normal(size=shape, dtype=np.float64)
+_BLOCK_ELEMS = 1 << 22
+_TAGS = {"q": 1, "k": 2, "v": 3, "gate": 4, "beta": 5, "state": 6}
+
+
+def _pool():
+    import concurrent.futures
+    import os
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:  # pragma: no cover
+        n = os.cpu_count() or 1
+    return concurrent.futures.ThreadPoolExecutor(max_workers=max(1, min(n, 32)))
+
+
+def _blocked(seed: int, tag: str, shape: tuple, transform, out_dtypes):
+    """Draw N(0,1) fp64 for ``shape`` block by block, map each block through
+    ``transform`` (fp64 block -> tuple of arrays) and assemble the outputs."""
+    shape = tuple(int(x) for x in shape)
+    rows = shape[0]
+    row_elems = int(np.prod(shape[1:])) if len(shape) > 1 else 1
+    per = max(1, _BLOCK_ELEMS // max(row_elems, 1))
+    outs = [np.empty(shape, dtype=dt) for dt in out_dtypes]
+
+    def work(b):
+        r0, r1 = b * per, min(rows, (b + 1) * per)
+        rng = np.random.default_rng([seed, _TAGS[tag], b])
+        x = rng.standard_normal(size=(r1 - r0,) + shape[1:], dtype=np.float64)
+        for o, y in zip(outs, transform(x)):
+            o[r0:r1] = y
+
+    nblk = (rows + per - 1) // per
+    if nblk <= 1:
+        for b in range(nblk):
+            work(b)
+    else:
+        with _pool() as ex:
+            list(ex.map(work, range(nblk)))
+    return outs
 
 
 def _unit_rows(x: np.ndarray) -> np.ndarray:
-    n = np.sqrt(np.sum(x * x, axis=-1, keepdims=True))
+    n = np.sqrt(np.einsum("...i,...i->...", x, x))[..., None]
     return x / n
 
 
@@ -178,31 +217,49 @@ def _sigmoid(x: np.ndarray) -> np.ndarray:
     return 1.0 / (1.0 + np.exp(-x))
 
 
-def _store(x64: np.ndarray, io_dtype: str):
-    """Return (stored array, exact float32 view of the stored values)."""
-    if io_dtype == "bf16":
-        bits = bf16_round(x64.astype(np.float32))
-        return bits, bf16_bits_to_f32(bits)
-    if io_dtype == "f32":
-        f = x64.astype(np.float32)
-        return f, f
-    raise ValueError(f"unknown io dtype {io_dtype}")
+def _io_transform(io_dtype: str, normalise: bool):
+    def f(x):
+        if normalise:
+            x = _unit_rows(x)
+        x32 = x.astype(np.float32)
+        if io_dtype == "bf16":
+            bits = bf16_round(x32)
+            return bits, bf16_bits_to_f32(bits)
+        if io_dtype == "f32":
+            return x32, x32
+        raise ValueError(f"unknown io dtype {io_dtype}")
+    return f
 
 
-def _draw_block(rng, w: Workload, lead: tuple):
-    """Draw q, k, v, gate, beta for token-axis shape ``lead`` (in that order)."""
-    q = _store(_unit_rows(_normal(rng, lead + (w.H_qk, w.d_k))), w.io_dtype)
-    k = _store(_unit_rows(_normal(rng, lead + (w.H_qk, w.d_k))), w.io_dtype)
-    v = _store(_normal(rng, lead + (w.H_v, w.d_v)), w.io_dtype)
+def _io_dtypes(io_dtype: str):
+    return (np.uint16, np.float32) if io_dtype == "bf16" else (np.float32, np.float32)
+
+
+def _draw_block(seed, w: Workload, lead: tuple):
+    """Draw q, k, v, gate, beta for token-axis shape ``lead``."""
+    io_t = _io_dtypes(w.io_dtype)
+    q, q32 = _blocked(seed, "q", lead + (w.H_qk, w.d_k), _io_transform(w.io_dtype, True), io_t)
+    k, k32 = _blocked(seed, "k", lead + (w.H_qk, w.d_k), _io_transform(w.io_dtype, True), io_t)
+    v, v32 = _blocked(seed, "v", lead + (w.H_v, w.d_v), _io_transform(w.io_dtype, False), io_t)
     if w.gate == "channel":
         gshape = lead + (w.H_v, w.d_k)
     elif w.gate == "scalar":
         gshape = lead + (w.H_v,)
     else:
         raise ValueError(w.gate)
-    g = (-w.gate_scale * _softplus(_normal(rng, gshape))).astype(np.float32)
-    beta = _sigmoid(_normal(rng, lead + (w.H_v,))).astype(np.float32)
-    return q, k, v, g, beta
+    if q is q32:
+        q32, k32, v32 = q, k, v
+    (g,) = _blocked(seed, "gate", gshape,
+                    lambda x: ((-w.gate_scale * _softplus(x)).astype(np.float32),), (np.float32,))
+    (beta,) = _blocked(seed, "beta", lead + (w.H_v,),
+                       lambda x: (_sigmoid(x).astype(np.float32),), (np.float32,))
+    return (q, q32), (k, k32), (v, v32), g, beta
+
+
+def _draw_state(seed, n, w: Workload):
+    (s0,) = _blocked(seed, "state", (n, w.H_v, w.d_k, w.d_v),
+                     lambda x: ((0.02 * x).astype(np.float32),), (np.float32,))
+    return s0
 
 
 def varlen_lengths(w: Workload, seed: int = 0) -> np.ndarray:
@@ -219,10 +276,8 @@ def make_prefill(w: Workload, seed: int = 0, lengths=None) -> PrefillInputs:
     """
     if w.kind != "prefill":
         raise ValueError("not a prefill workload")
-    rng = np.random.default_rng(seed)
     if lengths is None and w.varlen:
-        lo, hi = w.varlen_range
-        lengths = rng.integers(lo, hi, size=w.varlen, endpoint=True)
+        lengths = varlen_lengths(w, seed)
     if lengths is not None:
         lengths = np.asarray(lengths, dtype=np.int64)
         cu = np.zeros(len(lengths) + 1, dtype=np.int32)
@@ -231,10 +286,8 @@ def make_prefill(w: Workload, seed: int = 0, lengths=None) -> PrefillInputs:
         cu = (np.arange(w.B + 1, dtype=np.int64) * w.T).astype(np.int32)
     total = int(cu[-1])
     n = len(cu) - 1
-    (q, q32), (k, k32), (v, v32), g, beta = _draw_block(rng, w, (total,))
-    s0 = None
-    if w.init_state:
-        s0 = (0.02 * _normal(rng, (n, w.H_v, w.d_k, w.d_v))).astype(np.float32)
+    (q, q32), (k, k32), (v, v32), g, beta = _draw_block(seed, w, (total,))
+    s0 = _draw_state(seed, n, w) if w.init_state else None
     return PrefillInputs(w=w, q=q, k=k, v=v, g=g, beta=beta, initial_state=s0,
                          cu_seqlens=cu, q32=q32, k32=k32, v32=v32)
 
@@ -242,10 +295,9 @@ def make_prefill(w: Workload, seed: int = 0, lengths=None) -> PrefillInputs:
 def make_decode(w: Workload, seed: int = 0) -> DecodeInputs:
     if w.kind != "decode":
         raise ValueError("not a decode workload")
-    rng = np.random.default_rng(seed)
-    (q, q32), (k, k32), (v, v32), g, beta = _draw_block(rng, w, (w.steps, w.N))
+    (q, q32), (k, k32), (v, v32), g, beta = _draw_block(seed, w, (w.steps, w.N))
     if w.init_state:
-        s0 = (0.02 * _normal(rng, (w.N, w.H_v, w.d_k, w.d_v))).astype(np.float32)
+        s0 = _draw_state(seed, w.N, w)
     else:
         s0 = np.zeros((w.N, w.H_v, w.d_k, w.d_v), dtype=np.float32)
     return DecodeInputs(w=w, q=q, k=k, v=v, g=g, beta=beta, initial_state=s0,

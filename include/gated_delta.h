@@ -1,0 +1,169 @@
+/*
+ * gated_delta.h -- C ABI of the B200 (sm_100a) gated delta-rule library.
+ *
+ * The operator (thethings.ai, "The argument, in one page", table "Everything,
+ * in one table", rows "KDA" and "Gated DeltaNet"), with column-vector keys:
+ *
+ *     S_t = Diag(a_t) (I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+ *     o_t = S_t^T q_t
+ *
+ * S_t is a d_k x d_v fp32 state per (sequence, head), stored row-major
+ * [d_k][d_v] (row i belongs to key channel i).  a_t = exp(g_t) with g_t <= 0 a
+ * log-decay: a vector over d_k channels for KDA ("kda_*"), one scalar per
+ * (token, head) for Gated DeltaNet ("gdn_*").  The decay multiplies the state
+ * after the rank-one erase; the fresh write beta_t k_t v_t^T is not decayed
+ * (the operator order of the table rows).  o_t reads the state after token t's
+ * own update; there is no normaliser and no 1/sqrt(d_k) scale: q is used as
+ * given.
+ *
+ * General conventions
+ * -------------------
+ *  - Every data pointer is a DEVICE pointer owned by the caller; the library
+ *    allocates no device memory and keeps no state between calls except a
+ *    per-device cache of attributes.  Work is enqueued on `stream` (a
+ *    cudaStream_t; NULL = the legacy default stream) and the call returns
+ *    without synchronising.
+ *  - Token layout is [B, T, H, d] with d contiguous (equivalently [B*T, H, d]);
+ *    for packed variable-length batches B must be 1 and T is the total token
+ *    count.  g is [B, T, H_v, d_k] (KDA) or [B, T, H_v] (GDN); beta is
+ *    [B, T, H_v]; states are [N, H_v, d_k, d_v] where N is the number of
+ *    sequences (B, or num_seqs when cu_seqlens is given).
+ *  - q/k/v/o element type is io_dtype (KDA_BF16 or KDA_F32); g, beta and the
+ *    states are always fp32.  io_dtype = KDA_F32 selects the all-fp32 path.
+ *  - Supported head sizes: d_k in {64, 128}, d_v in {64, 128}.
+ *  - o must not alias any input.  All pointers must be 16-byte aligned.
+ *  - The return value reports host-side validation and launch errors.  Errors
+ *    found on the device (an invalid cu_seqlens array) are recorded in the
+ *    workspace and reported by kda_check_device_status().
+ *  - Thread safety: calls on different streams with disjoint buffers may run
+ *    concurrently.
+ */
+#ifndef GATED_DELTA_H
+#define GATED_DELTA_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KDA_ABI_VERSION 1
+
+#if defined(__GNUC__)
+#define KDA_API __attribute__((visibility("default")))
+#else
+#define KDA_API
+#endif
+
+typedef enum {
+  KDA_OK = 0,
+  KDA_ERR_INVALID_ARG = 1,   /* bad pointer, shape, alignment or size           */
+  KDA_ERR_UNSUPPORTED = 2,   /* valid but not implemented (e.g. d_k = 96)       */
+  KDA_ERR_CUDA = 3,          /* a CUDA runtime call or a launch failed          */
+  KDA_ERR_DEVICE_CHECK = 4,  /* a device-side check failed (see check call)     */
+  KDA_ERR_WORKSPACE = 5      /* workspace pointer NULL or smaller than required */
+} kda_status_t;
+
+typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
+
+/* Device-side error codes written to the workspace status word. */
+#define KDA_DEVICE_OK 0
+#define KDA_DEVICE_BAD_CU_SEQLENS 1  /* cu[0] != 0, decreasing, or cu[N] != T */
+
+/* --------------------------------------------------------------------------
+ * Prefill, per-channel gate (KDA).  Chunked over tokens; the state is carried
+ * across chunks on chip.  Row "KDA" of the table; the chunkwise computation
+ * follows row "Chunkwise / WY" (the result is the recurrence's, whatever the
+ * chunk size).
+ *
+ *   q, k          [B, T, H, d_k]   io_dtype
+ *   v             [B, T, H, d_v]   io_dtype
+ *   g             [B, T, H, d_k]   fp32 log-decay (<= 0; a = exp(g)).  The
+ *                                  bf16 path needs g >= -5 per token for the
+ *                                  sub-chunk scale factors to stay in range.
+ *   beta          [B, T, H]        fp32 write strength
+ *   o             [B, T, H, d_v]   io_dtype, written
+ *   initial_state [N, H, d_k, d_v] fp32, or NULL for zeros
+ *   final_state   [N, H, d_k, d_v] fp32, written, or NULL
+ *   cu_seqlens    [num_seqs + 1]   int32 DEVICE array of token offsets, or NULL
+ *                                  (then N = B dense sequences of T tokens).
+ *                                  Must satisfy cu[0] = 0, cu[i] <= cu[i+1],
+ *                                  cu[num_seqs] = T; zero-length sequences are
+ *                                  allowed (their final state = initial state).
+ *   workspace     device scratch of at least kda_chunk_fwd_workspace_size()
+ *                 bytes, 256-byte aligned; its contents are overwritten.
+ * ------------------------------------------------------------------------ */
+KDA_API kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, void *o, const float *initial_state,
+                           float *final_state, const int32_t *cu_seqlens, int32_t num_seqs,
+                           int32_t B, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                           kda_dtype_t io_dtype, void *workspace, size_t workspace_bytes,
+                           void *stream);
+
+KDA_API size_t kda_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                    int32_t num_seqs, kda_dtype_t io_dtype);
+
+/* --------------------------------------------------------------------------
+ * Prefill, scalar gate (Gated DeltaNet; row "Gated DeltaNet" of the table).
+ * q and k have H_qk heads; v, o, g, beta and the states have H_v heads, with
+ * H_v % H_qk == 0 and v-head h reading q/k head h / (H_v / H_qk).
+ *
+ *   q, k [B, T, H_qk, d_k]; v, o [B, T, H_v, d_v]; g, beta [B, T, H_v];
+ *   states [N, H_v, d_k, d_v].  Everything else as kda_chunk_fwd.
+ * ------------------------------------------------------------------------ */
+KDA_API kda_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
+                           const float *beta, void *o, const float *initial_state,
+                           float *final_state, const int32_t *cu_seqlens, int32_t num_seqs,
+                           int32_t B, int32_t T, int32_t H_qk, int32_t H_v, int32_t d_k,
+                           int32_t d_v, kda_dtype_t io_dtype, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+KDA_API size_t gdn_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H_qk, int32_t H_v,
+                                    int32_t d_k, int32_t d_v, int32_t num_seqs,
+                                    kda_dtype_t io_dtype);
+
+/* --------------------------------------------------------------------------
+ * One decode step, per-channel gate: one token for each of N sequences; the
+ * state is read once and updated IN PLACE.  Same operator as kda_chunk_fwd
+ * (inferencex.semianalysis.com "Linear attention": a recurrent state of
+ * constant size updated as tokens arrive).
+ *
+ *   q, k  [N, H, d_k] io_dtype;  v [N, H, d_v] io_dtype
+ *   g     [N, H, d_k] fp32 log-decay;  beta [N, H] fp32
+ *   o     [N, H, d_v] io_dtype, written
+ *   state [N, H, d_k, d_v] fp32, read and overwritten
+ * Needs no workspace.
+ * ------------------------------------------------------------------------ */
+KDA_API kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, void *o, float *state, int32_t N, int32_t H,
+                             int32_t d_k, int32_t d_v, kda_dtype_t io_dtype, void *stream);
+
+/* One decode step, scalar gate, q/k heads shared as in gdn_chunk_fwd:
+ *   q, k [N, H_qk, d_k]; v, o [N, H_v, d_v]; g, beta [N, H_v];
+ *   state [N, H_v, d_k, d_v] in place. */
+KDA_API kda_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
+                             const float *beta, void *o, float *state, int32_t N,
+                             int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+                             kda_dtype_t io_dtype, void *stream);
+
+/* Wait for `stream`, then read the device status word of a prefill workspace.
+ * Returns KDA_OK or KDA_ERR_DEVICE_CHECK (device code in *device_code when
+ * non-NULL), or KDA_ERR_CUDA.  Synchronises the stream. */
+KDA_API kda_status_t kda_check_device_status(const void *workspace, void *stream,
+                                     int32_t *device_code);
+
+/* Static text for a status code. */
+KDA_API const char *kda_status_string(kda_status_t status);
+
+/* Detail of the last error raised on the calling host thread ("" if none). */
+KDA_API const char *kda_last_error(void);
+
+/* KDA_ABI_VERSION of the loaded library. */
+KDA_API int32_t kda_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* GATED_DELTA_H */

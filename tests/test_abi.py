@@ -1,0 +1,102 @@
+"""The C ABI library without a GPU: it loads, exports every symbol the header
+declares, and rejects bad arguments on the host before touching the device."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import gated_delta_rule_87_b200 as gdr
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared_symbols():
+    text = open(os.path.join(ROOT, "include", "gated_delta.h")).read()
+    return sorted(set(re.findall(r"KDA_API\s+[\w\s\*]+?\b(\w+)\s*\(", text)))
+
+
+def test_library_loads_and_reports_abi_version():
+    L = gdr.lib()
+    assert L.kda_abi_version() == 1
+
+
+def test_every_declared_symbol_is_exported():
+    declared = _declared_symbols()
+    assert len(declared) == len(gdr.EXPORTED_SYMBOLS)
+    assert set(declared) == set(gdr.EXPORTED_SYMBOLS)
+    L = ctypes.CDLL(gdr.library_path)
+    for name in declared:
+        assert hasattr(L, name), name
+
+
+def test_status_strings():
+    L = gdr.lib()
+    for code in range(6):
+        assert L.kda_status_string(code)
+    assert L.kda_status_string(99) == b"unknown status"
+
+
+def test_workspace_size_is_host_only_and_monotone():
+    L = gdr.lib()
+    a = L.kda_chunk_fwd_workspace_size(1, 4096, 32, 128, 128, 0, 1)
+    b = L.kda_chunk_fwd_workspace_size(1, 8192, 32, 128, 128, 0, 1)
+    assert 256 <= a <= b
+    c = L.gdn_chunk_fwd_workspace_size(1, 4096, 16, 32, 128, 128, 0, 1)
+    assert c == a
+
+
+FAKE = 0x10000  # never dereferenced: every call below fails validation first
+
+
+def _prefill(**over):
+    L = gdr.lib()
+    kw = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, o=FAKE + 4096, s0=None, sT=None,
+              cu=None, num_seqs=0, B=1, T=64, H=2, d_k=128, d_v=128, io=1, ws=FAKE,
+              ws_bytes=1 << 20)
+    kw.update(over)
+    return L.kda_chunk_fwd(kw["q"], kw["k"], kw["v"], kw["g"], kw["beta"], kw["o"], kw["s0"],
+                           kw["sT"], kw["cu"], kw["num_seqs"], kw["B"], kw["T"], kw["H"],
+                           kw["d_k"], kw["d_v"], kw["io"], kw["ws"], kw["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(q=None), gdr.KDA_ERR_INVALID_ARG),
+    (dict(B=0), gdr.KDA_ERR_INVALID_ARG),
+    (dict(d_k=96), gdr.KDA_ERR_UNSUPPORTED),
+    (dict(d_v=32), gdr.KDA_ERR_UNSUPPORTED),
+    (dict(io=7), gdr.KDA_ERR_INVALID_ARG),
+    (dict(k=FAKE + 2), gdr.KDA_ERR_INVALID_ARG),
+    (dict(o=FAKE), gdr.KDA_ERR_INVALID_ARG),
+    (dict(ws=None), gdr.KDA_ERR_WORKSPACE),
+    (dict(ws=FAKE + 16), gdr.KDA_ERR_WORKSPACE),
+    (dict(ws_bytes=16), gdr.KDA_ERR_WORKSPACE),
+    (dict(cu=FAKE, num_seqs=2, B=2), gdr.KDA_ERR_INVALID_ARG),
+])
+def test_prefill_rejects_bad_arguments_on_host(over, status):
+    assert _prefill(**over) == status
+    assert gdr.lib().kda_last_error()
+
+
+def test_gdn_rejects_indivisible_head_groups():
+    L = gdr.lib()
+    st = L.gdn_chunk_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 4096, None, None, None, 0,
+                         1, 64, 3, 4, 128, 128, 1, FAKE, 1 << 20, None)
+    assert st == gdr.KDA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("args,status", [
+    ((None,) + (FAKE,) * 6 + (4, 2, 128, 128, 1), gdr.KDA_ERR_INVALID_ARG),
+    ((FAKE,) * 7 + (4, 2, 96, 128, 1), gdr.KDA_ERR_UNSUPPORTED),
+    ((FAKE,) * 7 + (4, 2, 128, 128, 1), gdr.KDA_ERR_INVALID_ARG),  # o aliases the inputs
+    ((FAKE,) * 5 + (FAKE + 8,) + (FAKE,) + (4, 2, 128, 128, 1), gdr.KDA_ERR_INVALID_ARG),
+])
+def test_decode_rejects_bad_arguments_on_host(args, status):
+    L = gdr.lib()
+    assert L.kda_decode_step(*args, None) == status
+
+
+def test_binding_has_no_cpu_path():
+    """The product binding never imports the oracle."""
+    src = open(os.path.join(ROOT, "gated_delta_rule_87_b200", "__init__.py")).read()
+    assert "oracle" not in re.sub(r'""".*?"""', "", src, flags=re.S)

@@ -1,0 +1,163 @@
+"""Chunked prefill on the GPU against the fp64 oracle (same seeded inputs)."""
+import numpy as np
+import pytest
+
+from gated_delta_rule_87_b200 import workloads as W
+from parity import oracle_prefill, prefill_device_inputs, rel_l2, to_host, tol_for
+
+pytestmark = pytest.mark.gpu
+
+
+def _run(x, **kw):
+    import torch
+    import gated_delta_rule_87_b200 as gdr
+    d = prefill_device_inputs(x)
+    fn = gdr.kda_chunk_fwd if x.w.gate == "channel" else gdr.gdn_chunk_fwd
+    o, sT, ws = fn(d["q"], d["k"], d["v"], d["g"], d["beta"], d["initial_state"],
+                   d["cu_seqlens"], **kw)
+    torch.cuda.synchronize()
+    st, code = gdr.check_device_status(ws)
+    assert st == gdr.KDA_OK, code
+    o = to_host(o).reshape(x.total_tokens, x.w.H_v, x.w.d_v)
+    return o, sT.cpu().numpy()
+
+
+def _check(x, heads=None, tol=None):
+    o, sT = _run(x)
+    ro, rs = oracle_prefill(x, heads)
+    if heads is not None:
+        o, sT = o[:, heads], sT[:, heads]
+    tol = tol or tol_for(x.w.io_dtype)
+    eo, es = rel_l2(o, ro), rel_l2(sT, rs)
+    assert np.isfinite(o).all() and np.isfinite(sT).all()
+    assert eo <= tol, f"output rel-L2 {eo:.3e} > {tol}"
+    assert es <= tol, f"final-state rel-L2 {es:.3e} > {tol}"
+    return eo, es
+
+
+def test_gdn_small_fp32_workload():
+    """All-fp32 Gated DeltaNet, B=1 H=2 T=128 d=64, against the 1e-4 bound."""
+    x = W.make_prefill(W.WORKLOADS["gdn_small_f32"], seed=0)
+    _check(x)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+@pytest.mark.parametrize("T", [1, 17, 63, 64, 65, 130, 257])
+def test_kda_ragged_lengths(io, T):
+    w = W.WORKLOADS["kda_prefill"].replace(T=T, H_qk=2, H_v=2, io_dtype=io)
+    _check(W.make_prefill(w, seed=T))
+
+
+@pytest.mark.parametrize("dk,dv", [(64, 64), (64, 128), (128, 64)])
+def test_kda_head_sizes(dk, dv):
+    for io in ("f32", "bf16"):
+        w = W.WORKLOADS["kda_prefill"].replace(T=200, H_qk=2, H_v=2, d_k=dk, d_v=dv, io_dtype=io)
+        _check(W.make_prefill(w, seed=3))
+
+
+def test_kda_dense_batch():
+    w = W.WORKLOADS["kda_prefill"].replace(B=3, T=150, H_qk=2, H_v=2)
+    _check(W.make_prefill(w, seed=4))
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_kda_packed_with_empty_sequences(io):
+    w = W.WORKLOADS["kda_varlen"].replace(H_qk=2, H_v=2, io_dtype=io, init_state=True)
+    x = W.make_prefill(w, seed=5, lengths=[70, 0, 1, 128, 0, 200])
+    _check(x)
+
+
+@pytest.mark.parametrize("io", ["f32", "bf16"])
+def test_gdn_shared_heads(io):
+    w = W.WORKLOADS["gdn_long"].replace(T=300, H_qk=2, H_v=4, io_dtype=io, init_state=True)
+    _check(W.make_prefill(w, seed=6))
+
+
+def test_no_initial_state_no_final_state():
+    import torch
+    import gated_delta_rule_87_b200 as gdr
+    w = W.WORKLOADS["kda_prefill"].replace(T=100, H_qk=2, H_v=2, init_state=False)
+    x = W.make_prefill(w, seed=8)
+    d = prefill_device_inputs(x)
+    o, sT, _ = gdr.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None,
+                                 output_final_state=False)
+    torch.cuda.synchronize()
+    assert sT is None
+    ro, _ = oracle_prefill(x)
+    assert rel_l2(to_host(o).reshape(ro.shape), ro) <= 2e-2
+
+
+def test_split_prefill_carries_state():
+    """prefill(T1) then prefill(T2) from its final state == prefill(T1 + T2)."""
+    import torch
+    import gated_delta_rule_87_b200 as gdr
+    w = W.WORKLOADS["kda_prefill"].replace(T=320, H_qk=2, H_v=2)
+    x = W.make_prefill(w, seed=9)
+    d = prefill_device_inputs(x)
+    o, s, _ = gdr.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], d["initial_state"])
+    cut = 137
+    part = lambda t, a, b: t[:, a:b].contiguous()
+    o1, s1, _ = gdr.kda_chunk_fwd(*(part(d[n], 0, cut) for n in ("q", "k", "v", "g", "beta")),
+                                  d["initial_state"])
+    o2, s2, _ = gdr.kda_chunk_fwd(*(part(d[n], cut, 320) for n in ("q", "k", "v", "g", "beta")),
+                                  s1)
+    torch.cuda.synchronize()
+    full = to_host(o)
+    split = np.concatenate([to_host(o1), to_host(o2)], axis=1)
+    assert rel_l2(split, full) <= 1e-2
+    assert rel_l2(s2.cpu().numpy(), s.cpu().numpy()) <= 1e-2
+
+
+def test_decode_after_prefill_matches_longer_prefill():
+    """A prefill of T tokens followed by n decode steps equals one prefill of
+    T + n tokens (the state is the only carrier of the past)."""
+    import torch
+    import gated_delta_rule_87_b200 as gdr
+    w = W.WORKLOADS["kda_prefill"].replace(T=96, H_qk=2, H_v=2)
+    x = W.make_prefill(w, seed=10)
+    d = prefill_device_inputs(x)
+    T0 = 80
+    part = lambda t, a, b: t[:, a:b].contiguous()
+    _, s, _ = gdr.kda_chunk_fwd(*(part(d[n], 0, T0) for n in ("q", "k", "v", "g", "beta")),
+                                d["initial_state"])
+    outs = []
+    for t in range(T0, 96):
+        sl = lambda n: d[n][0, t].contiguous().unsqueeze(0)
+        outs.append(to_host(gdr.kda_decode_step(sl("q"), sl("k"), sl("v"), sl("g"), sl("beta"), s)))
+    torch.cuda.synchronize()
+    ro, rs = oracle_prefill(x)
+    assert rel_l2(np.concatenate(outs, axis=0), ro[T0:]) <= 2e-2
+    assert rel_l2(s.cpu().numpy(), rs) <= 2e-2
+
+
+def test_invalid_cu_seqlens_is_reported_on_device():
+    import torch
+    import gated_delta_rule_87_b200 as gdr
+    w = W.WORKLOADS["kda_varlen"].replace(H_qk=2, H_v=2)
+    x = W.make_prefill(w, seed=11, lengths=[64, 64])
+    d = prefill_device_inputs(x)
+    bad = torch.tensor([0, 80, 64], dtype=torch.int32, device="cuda")  # decreasing
+    o = torch.full_like(d["v"], float("nan"))
+    _, _, ws = gdr.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"], None, bad, o=o)
+    st, code = gdr.check_device_status(ws)
+    assert st == gdr.KDA_ERR_DEVICE_CHECK and code == 1
+
+
+# ----------------------------------------------------------------------------
+# the full workloads (the bench's launch configuration), sampled where the
+# oracle would take long
+# ----------------------------------------------------------------------------
+def test_kda_prefill_full_workload():
+    x = W.make_prefill(W.WORKLOADS["kda_prefill"], seed=0)
+    _check(x)
+
+
+def test_kda_varlen_full_workload_sampled_heads():
+    x = W.make_prefill(W.WORKLOADS["kda_varlen"], seed=0)
+    assert list(np.diff(x.cu_seqlens)) == [14090, 10808, 8875, 5168, 5752, 1653, 2179, 1277]
+    _check(x, heads=[0, 13, 31])
+
+
+def test_gdn_long_full_workload_sampled_heads():
+    x = W.make_prefill(W.WORKLOADS["gdn_long"], seed=0)
+    _check(x, heads=[0, 1, 30])
