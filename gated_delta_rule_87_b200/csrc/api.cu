@@ -29,6 +29,7 @@ kda_status_t cuda_fail(cudaError_t e, const char *where) {
 }
 
 bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+bool aligned4(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 3u) == 0; }
 
 bool head_dim_ok(int d) { return d == 64 || d == 128; }
 
@@ -37,7 +38,8 @@ constexpr size_t kStatusBytes = 256;
 
 // Validation shared by both prefill entry points.
 kda_status_t check_prefill(const gdr::PrefillArgs &a) {
-  if (!a.q || !a.k || !a.v || !a.g || !a.beta || !a.o)
+  const bool empty = (int64_t)a.B * a.T == 0;  // no tokens: data pointers may be NULL
+  if (!empty && (!a.q || !a.k || !a.v || !a.g || !a.beta || !a.o))
     return fail(KDA_ERR_INVALID_ARG, "q, k, v, g, beta and o must be non-NULL");
   if (a.B <= 0 || a.T < 0 || a.H_qk <= 0 || a.H_v <= 0)
     return fail(KDA_ERR_INVALID_ARG, "need B > 0, T >= 0, H > 0 (B=%d T=%d H_qk=%d H_v=%d)", a.B,
@@ -46,17 +48,18 @@ kda_status_t check_prefill(const gdr::PrefillArgs &a) {
     return fail(KDA_ERR_INVALID_ARG, "H_v (%d) must be a multiple of H_qk (%d)", a.H_v, a.H_qk);
   if (!head_dim_ok(a.d_k) || !head_dim_ok(a.d_v))
     return fail(KDA_ERR_UNSUPPORTED, "d_k and d_v must be 64 or 128 (got %d, %d)", a.d_k, a.d_v);
-  const void *ptrs[] = {a.q, a.k, a.v, a.g, a.beta, a.o, a.initial_state, a.final_state,
-                        a.cu_seqlens};
-  for (const void *p : ptrs)
+  const void *ptrs16[] = {a.q, a.k, a.v, a.g, a.o, a.initial_state, a.final_state};
+  for (const void *p : ptrs16)
     if (p && !aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", p);
+  if ((a.beta && !aligned4(a.beta)) || (a.cu_seqlens && !aligned4(a.cu_seqlens)))
+    return fail(KDA_ERR_INVALID_ARG, "beta and cu_seqlens must be 4-byte aligned");
   if (a.cu_seqlens) {
     if (a.B != 1) return fail(KDA_ERR_INVALID_ARG, "packed sequences (cu_seqlens) need B == 1");
     if (a.num_seqs < 0) return fail(KDA_ERR_INVALID_ARG, "num_seqs must be >= 0");
   }
   if ((int64_t)a.B * a.T > INT32_MAX)
     return fail(KDA_ERR_INVALID_ARG, "B*T must fit in int32");
-  if (a.o == a.q || a.o == a.k || a.o == a.v)
+  if (!empty && (a.o == a.q || a.o == a.k || a.o == a.v))
     return fail(KDA_ERR_INVALID_ARG, "o must not alias q, k or v");
   if (!a.workspace) return fail(KDA_ERR_WORKSPACE, "workspace is NULL");
   if (reinterpret_cast<uintptr_t>(a.workspace) & 255u)
@@ -197,6 +200,7 @@ static kda_status_t decode_common(gdr::DecodeArgs &a, kda_dtype_t io_dtype, void
   if (io_dtype != KDA_F32 && io_dtype != KDA_BF16)
     return fail(KDA_ERR_INVALID_ARG, "io_dtype must be KDA_F32 or KDA_BF16");
   a.bf16 = (io_dtype == KDA_BF16);
+  if (a.N == 0 && a.H_qk > 0 && a.H_v > 0) return KDA_OK;  // empty batch: nothing to do
   if (!a.q || !a.k || !a.v || !a.g || !a.beta || !a.o || !a.state)
     return fail(KDA_ERR_INVALID_ARG, "q, k, v, g, beta, o and state must be non-NULL");
   if (a.N < 0 || a.H_qk <= 0 || a.H_v <= 0)
@@ -207,9 +211,15 @@ static kda_status_t decode_common(gdr::DecodeArgs &a, kda_dtype_t io_dtype, void
     return fail(KDA_ERR_UNSUPPORTED, "d_k and d_v must be 64 or 128 (got %d, %d)", a.d_k, a.d_v);
   if ((int64_t)a.N * a.H_v > INT32_MAX)
     return fail(KDA_ERR_INVALID_ARG, "N*H must fit in int32");
-  const void *ptrs[] = {a.q, a.k, a.v, a.g, a.beta, a.o, a.state};
+  if (!aligned16(a.state))
+    return fail(KDA_ERR_INVALID_ARG, "state %p is not 16-byte aligned", (const void *)a.state);
+  const size_t esz = a.bf16 ? 2 : 4;
+  const void *ptrs[] = {a.q, a.k, a.v, a.o};
   for (const void *p : ptrs)
-    if (!aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", p);
+    if (reinterpret_cast<uintptr_t>(p) % esz)
+      return fail(KDA_ERR_INVALID_ARG, "pointer %p is not aligned to its element size", p);
+  if (!aligned4(a.g) || !aligned4(a.beta))
+    return fail(KDA_ERR_INVALID_ARG, "g and beta must be 4-byte aligned");
   if (a.o == a.q || a.o == a.k || a.o == a.v || a.o == a.state)
     return fail(KDA_ERR_INVALID_ARG, "o must not alias an input or the state");
   cudaError_t e = gdr::launch_decode_step(a, static_cast<cudaStream_t>(stream));

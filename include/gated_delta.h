@@ -31,7 +31,9 @@
  *  - q/k/v/o element type is io_dtype (KDA_BF16 or KDA_F32); g, beta and the
  *    states are always fp32.  io_dtype = KDA_F32 selects the all-fp32 path.
  *  - Supported head sizes: d_k in {64, 128}, d_v in {64, 128}.
- *  - o must not alias any input.  All pointers must be 16-byte aligned.
+ *  - o must not alias any input.  Prefill: q, k, v, g, o and the states must
+ *    be 16-byte aligned, beta and cu_seqlens 4-byte aligned.  Decode: the
+ *    state 16-byte aligned, the others aligned to their element size.
  *  - The return value reports host-side validation and launch errors.  Errors
  *    found on the device (an invalid cu_seqlens array) are recorded in the
  *    workspace and reported by kda_check_device_status().

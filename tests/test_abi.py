@@ -89,7 +89,9 @@ def test_gdn_rejects_indivisible_head_groups():
     ((None,) + (FAKE,) * 6 + (4, 2, 128, 128, 1), gdr.KDA_ERR_INVALID_ARG),
     ((FAKE,) * 7 + (4, 2, 96, 128, 1), gdr.KDA_ERR_UNSUPPORTED),
     ((FAKE,) * 7 + (4, 2, 128, 128, 1), gdr.KDA_ERR_INVALID_ARG),  # o aliases the inputs
-    ((FAKE,) * 5 + (FAKE + 8,) + (FAKE,) + (4, 2, 128, 128, 1), gdr.KDA_ERR_INVALID_ARG),
+    ((FAKE,) * 5 + (FAKE + 8,) + (FAKE + 8,) + (4, 2, 128, 128, 1), gdr.KDA_ERR_INVALID_ARG),
+    ((FAKE,) * 3 + (FAKE + 2,) + (FAKE,) + (FAKE + 4096,) + (FAKE + 8192,) + (4, 2, 128, 128, 1),
+     gdr.KDA_ERR_INVALID_ARG),
 ])
 def test_decode_rejects_bad_arguments_on_host(args, status):
     L = gdr.lib()
