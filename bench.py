@@ -72,6 +72,42 @@ def prefill_flops(w: W.Workload, total_tokens: int, C: int = 64) -> float:
     return float(total_tokens) * w.H_v * (7 * C * d + 6 * d * d)
 
 
+def kernel_algo_bytes(name: str, w: W.Workload, total_tokens: int, num_seqs: int) -> int:
+    """Algorithmic bytes one launch of a library kernel must move.
+
+    chunk_prep_kernel reads every input token once (q, k, v, gate, beta);
+    chunk_scan_kernel writes o and reads/writes the states; the single-kernel
+    fp32 path moves everything."""
+    e = 2 if w.io_dtype == "bf16" else 4
+    gate = 4 * w.H_v * (w.d_k if w.gate == "channel" else 1)
+    states = (2 if w.init_state else 1) * num_seqs * w.H_v * w.d_k * w.d_v * 4
+    if name.startswith("chunk_prep"):
+        return total_tokens * ((2 * w.H_qk * w.d_k + w.H_v * w.d_v) * e + gate + 4 * w.H_v)
+    if name.startswith("chunk_scan"):
+        return total_tokens * w.H_v * w.d_v * e + states
+    if name.startswith("plan"):
+        return 4 * (num_seqs + 1)
+    return prefill_bytes(w, total_tokens, num_seqs)
+
+
+def measured_traffic(kernel: str, workload: str):
+    """DRAM bytes (read + write) per launch from a committed ncu summary, or
+    None if the kernel's source changed since the counters were taken."""
+    import hashlib
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel, {}).get(workload)
+        if not rec:
+            return None
+        src = os.path.join(ROOT, rec["source"])
+        with open(src, "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()[:16]
+        return rec["bytes"] if sha == rec["source_sha256_16"] else None
+    except Exception:
+        return None
+
+
 def decode_bytes_per_head(w: W.Workload) -> int:
     e = 2 if w.io_dtype == "bf16" else 4
     return 2 * w.d_k * w.d_v * 4 + (2 * w.d_k + 2 * w.d_v) * e + 4 * w.d_k + 4
@@ -81,61 +117,60 @@ def decode_bytes_per_head(w: W.Workload) -> int:
 # clocks during the timed region
 # --------------------------------------------------------------------------- #
 class ClockSampler:
-    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
-              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
-              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    """Samples SM clocks and throttle reasons (NVML, every ~2 ms) while the
+    timed region runs.  Reads settings only."""
+
+    REASONS = {  # NVML clocks-event-reason bits
+        "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+        "sw_power_cap": 0x4, "hw_power_brake_slowdown": 0x80,
+    }
 
     def __init__(self, gpu_index: int):
         self.gpu = gpu_index
-        self.proc = None
-        self.lines = []
-        self.thread = None
+        self.samples = []
+        self.reasons = set()
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self._nv = None
 
     def __enter__(self):
         try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
-            self.thread = threading.Thread(target=self._read, daemon=True)
-            self.thread.start()
+            import pynvml as nv
+            nv.nvmlInit()
+            self._nv = nv
+            self._h = nv.nvmlDeviceGetHandleByIndex(self.gpu)
+            self.max_mhz = nv.nvmlDeviceGetMaxClockInfo(self._h, nv.NVML_CLOCK_SM)
+            self._thread = threading.Thread(target=self._run, daemon=True)
+            self._thread.start()
         except Exception:
-            self.proc = None
+            self._nv = None
         return self
 
-    def _read(self):
-        for line in self.proc.stdout:
-            self.lines.append(line.strip())
+    def _run(self):
+        nv = self._nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self._h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self._h)
+                for name, bit in self.REASONS.items():
+                    if bits & bit:
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(0.002)
 
     def __exit__(self, *exc):
-        if self.proc is not None:
-            self.proc.terminate()
-            try:
-                self.proc.wait(timeout=5)
-            except Exception:
-                self.proc.kill()
-            if self.thread:
-                self.thread.join(timeout=2)
+        self._stop.set()
+        if self._thread is not None:
+            self._thread.join(timeout=2)
 
     def summary(self):
-        sm, smax, reasons = [], [], set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
-            parts = [p.strip() for p in ln.split(",")]
-            if len(parts) < 9:
-                continue
-            try:
-                sm.append(float(parts[1]))
-                smax.append(float(parts[2]))
-            except ValueError:
-                continue
-            for nm, val in zip(names, parts[5:9]):
-                if val.lower() == "active":
-                    reasons.add(nm)
-        if not sm:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["unavailable"], "samples": 0}
-        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
-                "reasons": sorted(reasons), "samples": len(sm)}
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": ["unavailable"],
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
 
 
 # --------------------------------------------------------------------------- #
@@ -148,20 +183,31 @@ def dist_setup():
     return world, rank, local
 
 
-def max_over_ranks(x: float, world: int, device) -> float:
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """Max of a per-rank scalar over all ranks (CPU tensor under gloo)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device=device)
+    on_cpu = dist.get_backend() == "gloo" or device is None
+    t = torch.tensor([x], dtype=torch.float64, device="cpu" if on_cpu else device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
 
 
-def barrier(world: int, device):
+def barrier(world: int, device=None):
     if world > 1:
         import torch.distributed as dist
-        dist.barrier(device_ids=[device.index])
+        if dist.get_backend() == "gloo" or device is None:
+            dist.barrier()
+        else:
+            dist.barrier(device_ids=[device.index])
+
+
+def aggregate_throughput(units_per_rank: float, ms_max: float, world: int) -> float:
+    """Whole-job throughput of weakly scaled replicas: every rank processes
+    its own ``units_per_rank``; the job takes as long as the slowest rank."""
+    return units_per_rank * world / (ms_max / 1e3)
 
 
 # --------------------------------------------------------------------------- #
@@ -236,19 +282,42 @@ def run_ours(args, world, rank, local):
     ms_local = sum(per) / len(per)
     ms = max_over_ranks(ms_local, world, device)
     tokens = T_total
-    value = tokens * world / (ms / 1e3)
+    value = aggregate_throughput(tokens, ms, world)
+
+    # ---- per-kernel device times: the same calls again, with launch tracing ----
+    gdr.trace_enable(True)
+    for i in range(args.steps):
+        flush.zero_()
+        step(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], s0)
+    torch.cuda.synchronize()
+    recs = gdr.trace_read()
+    gdr.trace_enable(False)
+    per_kernel = {}
+    for name, t in recs:
+        per_kernel.setdefault(name, []).append(t)
+    kern_ms = {k: sum(v) / len(v) for k, v in per_kernel.items()}
+    dominant = max(kern_ms, key=kern_ms.get)
 
     algo_bytes = prefill_bytes(w, T_total, N)
     algo_flops = prefill_flops(w, T_total)
-    achieved_gbs = algo_bytes / (ms_local / 1e3) / 1e9
-    roofline = {"bound": "hbm", "achieved": round(achieved_gbs, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved_gbs / peaks["hbm_gbs"], 4),
-                "traffic": None, "peak_source": peaks["source"],
-                "kernel": "prefill (whole call)",
-                "achieved_tflops": round(algo_flops / (ms_local / 1e3) / 1e12, 2),
-                "roofline_tokens_per_s": round(tokens / max(algo_bytes / (peaks["hbm_gbs"] * 1e9),
-                                                           algo_flops / (peaks["bf16_tflops"] * 1e12)),
-                                               1)}
+    kb = kernel_algo_bytes(dominant, w, T_total, N)
+    achieved = kb / (kern_ms[dominant] / 1e3) / 1e9
+    traffic = measured_traffic(dominant, w.name)
+    roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": traffic, "peak_source": peaks["source"], "kernel": dominant,
+                "kernel_us": round(kern_ms[dominant] * 1e3, 2), "algorithmic_bytes": kb}
+    call_gbs = algo_bytes / (ms_local / 1e3) / 1e9
+    t_roof = max(algo_bytes / (peaks["hbm_gbs"] * 1e9), algo_flops / (peaks["bf16_tflops"] * 1e12))
+    call_roofline = {"bound": "hbm" if algo_bytes / peaks["hbm_gbs"] >= algo_flops / peaks["bf16_tflops"] / 1e3 else "tensor",
+                     "algorithmic_bytes": algo_bytes, "algorithmic_flops": algo_flops,
+                     "achieved_gbs": round(call_gbs, 1),
+                     "achieved_tflops": round(algo_flops / (ms_local / 1e3) / 1e12, 2),
+                     "roofline_us": round(t_roof * 1e6, 2),
+                     "frac": round(t_roof / (ms_local / 1e3), 4),
+                     "roofline_tokens_per_s": round(tokens / t_roof, 1)}
+    kernels = {k: {"us": round(v * 1e3, 2), "launches_per_step": len(per_kernel[k]) // args.steps}
+               for k, v in kern_ms.items()}
 
     # ---- end to end through the public API: pinned host -> device, call, back ----
     o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
@@ -287,6 +356,8 @@ def run_ours(args, world, rank, local):
                    "l2": "flushed (256 MB write) before every timed call",
                    "parallelism": f"replicas x{world}, no collective"},
         "roofline": roofline,
+        "call_roofline": call_roofline,
+        "kernels": kernels,
         "e2e": {"value": round(tokens * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
                 "d2h_bytes_per_step": d2h},
@@ -311,14 +382,13 @@ def run_ours(args, world, rank, local):
 
 
 def gdr_launches_per_call(w: W.Workload, varlen: bool) -> int:
-    """Our kernels per prefill call: the prefill kernel(s), plus the cu_seqlens
-    check for packed batches (the status reset is a memset, not a kernel)."""
+    """Our kernels per prefill call.  Tensor-core path (bf16, d = 128): plan,
+    prep and scan.  fp32 path: the chunk kernel, plus the cu_seqlens check for
+    packed batches.  (The status reset is a memset, not a kernel.)"""
     tc = w.io_dtype == "bf16" and w.d_k == 128 and w.d_v == 128
-    n = 2 if (tc and TC_TWO_PHASE) else 1
-    return n + (1 if varlen else 0)
-
-
-TC_TWO_PHASE = False
+    if tc:
+        return 3
+    return 1 + (1 if varlen else 0)
 
 
 def bench_decode(args, device, world, peaks, stream, flush):

@@ -22,6 +22,7 @@ from typing import Optional, Tuple
 __all__ = [
     "lib", "library_path", "KdaError", "kda_chunk_fwd", "gdn_chunk_fwd", "kda_decode_step",
     "gdn_decode_step", "chunk_workspace_size", "check_device_status", "EXPORTED_SYMBOLS",
+    "trace_enable", "trace_read",
     "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
     "KDA_ERR_DEVICE_CHECK", "KDA_ERR_WORKSPACE",
 ]
@@ -37,6 +38,7 @@ EXPORTED_SYMBOLS = (
     "kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "gdn_chunk_fwd",
     "gdn_chunk_fwd_workspace_size", "kda_decode_step", "gdn_decode_step",
     "kda_check_device_status", "kda_status_string", "kda_last_error", "kda_abi_version",
+    "kda_trace_enable", "kda_trace_read",
 )
 
 _lock = threading.Lock()
@@ -54,6 +56,8 @@ _SIGS = {
     "kda_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "kda_last_error": ([], ctypes.c_char_p),
     "kda_abi_version": ([], _i32),
+    "kda_trace_enable": ([_i32], ctypes.c_int),
+    "kda_trace_read": ([ctypes.c_char_p, _i32, ctypes.POINTER(ctypes.c_float), _i32], _i32),
 }
 
 
@@ -232,6 +236,22 @@ def gdn_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):
     """One Gated DeltaNet decode step (scalar gate, q/k heads shared by groups of
     v heads); ``state`` is updated in place.  Returns o [N,H_v,d_v]."""
     return _decode("scalar", q, k, v, g, beta, state, o, stream)
+
+
+def trace_enable(on: bool = True) -> None:
+    """Record the device time of every library kernel launch (off by default)."""
+    lib().kda_trace_enable(1 if on else 0)
+
+
+def trace_read(capacity: int = 4096):
+    """Wait for the traced launches; return [(kernel name, ms), ...] and clear."""
+    L = lib()
+    stride = 64
+    names = ctypes.create_string_buffer(stride * capacity)
+    ms = (ctypes.c_float * capacity)()
+    n = L.kda_trace_read(names, stride, ms, capacity)
+    return [(names.raw[i * stride:(i + 1) * stride].split(b"\0", 1)[0].decode(), float(ms[i]))
+            for i in range(n)]
 
 
 def check_device_status(workspace, stream=None) -> Tuple[int, int]:

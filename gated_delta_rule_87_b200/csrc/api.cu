@@ -80,11 +80,11 @@ kda_status_t run_prefill(gdr::PrefillArgs &a, cudaStream_t s) {
   int32_t *status = reinterpret_cast<int32_t *>(a.workspace);
   cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
-  if (a.cu_seqlens) {
+  if (!a.cu_seqlens) a.num_seqs = a.B;
+  const bool tc = use_tensor_core_path(a);
+  if (a.cu_seqlens && !tc) {  // the tensor-core path validates in its planning kernel
     e = gdr::launch_check_cu_seqlens(a.cu_seqlens, a.num_seqs, a.T, status, s);
     if (e != cudaSuccess) return cuda_fail(e, "cu_seqlens check launch");
-  } else {
-    a.num_seqs = a.B;
   }
   if (a.num_seqs == 0 || a.T == 0) {
     // nothing to compute; final state = initial state
@@ -100,7 +100,7 @@ kda_status_t run_prefill(gdr::PrefillArgs &a, cudaStream_t s) {
     return KDA_OK;
   }
   a.max_chunks = (int64_t)(a.B * (int64_t)a.T) / gdr::kChunk + a.num_seqs;
-  e = use_tensor_core_path(a) ? gdr::launch_prefill_tc(a, s) : gdr::launch_prefill_f32(a, s);
+  e = tc ? gdr::launch_prefill_tc(a, s) : gdr::launch_prefill_f32(a, s);
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   return KDA_OK;
 }

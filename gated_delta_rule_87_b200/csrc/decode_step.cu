@@ -179,6 +179,7 @@ cudaError_t launch_io(const DecodeArgs &a, cudaStream_t s) {
 
 cudaError_t launch_decode_step(const DecodeArgs &a, cudaStream_t stream) {
   if (a.N == 0) return cudaSuccess;
+  TraceScope tr("decode_step_kernel", stream);
   if (a.bf16) return launch_io<__nv_bfloat16>(a, stream);
   return launch_io<float>(a, stream);
 }

@@ -7,6 +7,22 @@
 
 namespace gdr {
 
+// Records the device time of the enclosed launch(es) on `s` when tracing is
+// enabled (kda_trace_enable); does nothing otherwise.
+class TraceScope {
+ public:
+  TraceScope(const char *name, cudaStream_t s);
+  ~TraceScope();
+  TraceScope(const TraceScope &) = delete;
+  TraceScope &operator=(const TraceScope &) = delete;
+
+ private:
+  const char *name_;
+  cudaStream_t stream_;
+  void *start_ = nullptr;
+  void *stop_ = nullptr;
+};
+
 struct DecodeArgs {
   const void *q, *k, *v;
   const float *g, *beta;

@@ -63,7 +63,6 @@ prefill_simt_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO
   extern __shared__ __align__(16) unsigned char smem_raw[];
   using Sm = SimtSmem<D_K>;
   Sm &sm = *reinterpret_cast<Sm *>(smem_raw);
-  constexpr int LD = Sm::LD;
 
   if (status && *status != KDA_DEVICE_OK) return;
 
@@ -235,6 +234,7 @@ cudaError_t launch_cfg(const PrefillArgs &a, cudaStream_t s) {
   if (e != cudaSuccess) return e;
   const unsigned grid = (unsigned)((int64_t)a.num_seqs * a.H_v * (D_V / NS));
   if (grid == 0) return cudaSuccess;
+  TraceScope tr("prefill_simt_kernel", s);
   kern<<<grid, kThreads, smem, s>>>((const IO *)a.q, (const IO *)a.k, (const IO *)a.v, a.g,
                                    a.beta, (IO *)a.o, a.initial_state, a.final_state,
                                    a.cu_seqlens, a.T, a.H_qk, a.H_v,

@@ -72,6 +72,7 @@ typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
 /* Device-side error codes written to the workspace status word. */
 #define KDA_DEVICE_OK 0
 #define KDA_DEVICE_BAD_CU_SEQLENS 1  /* cu[0] != 0, decreasing, or cu[N] != T */
+#define KDA_DEVICE_TIMEOUT 2         /* a bounded on-device wait expired */
 
 /* --------------------------------------------------------------------------
  * Prefill, per-channel gate (KDA).  Chunked over tokens; the state is carried
@@ -160,6 +161,15 @@ KDA_API const char *kda_status_string(kda_status_t status);
 
 /* Detail of the last error raised on the calling host thread ("" if none). */
 KDA_API const char *kda_last_error(void);
+
+/* Optional per-kernel device timing.  With kda_trace_enable(1), every kernel
+ * the library launches is bracketed by two CUDA events on the caller's stream
+ * (adds two event records per launch; off by default).  kda_trace_read()
+ * waits for the recorded launches, writes up to `capacity` kernel names
+ * (NUL-terminated, `name_stride` bytes apart) and durations in milliseconds,
+ * clears the record list and returns the number of records written. */
+KDA_API kda_status_t kda_trace_enable(int32_t on);
+KDA_API int32_t kda_trace_read(char *names, int32_t name_stride, float *ms, int32_t capacity);
 
 /* KDA_ABI_VERSION of the loaded library. */
 KDA_API int32_t kda_abi_version(void);
