@@ -38,7 +38,7 @@ EXPORTED_SYMBOLS = (
     "kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "gdn_chunk_fwd",
     "gdn_chunk_fwd_workspace_size", "kda_decode_step", "gdn_decode_step",
     "kda_check_device_status", "kda_status_string", "kda_last_error", "kda_abi_version",
-    "kda_trace_enable", "kda_trace_read",
+    "kda_trace_enable", "kda_trace_read", "kda_chunk_fwd_noalloc",
 )
 
 _lock = threading.Lock()
@@ -57,6 +57,7 @@ _SIGS = {
     "kda_last_error": ([], ctypes.c_char_p),
     "kda_abi_version": ([], _i32),
     "kda_trace_enable": ([_i32], ctypes.c_int),
+    "kda_chunk_fwd_noalloc": ([_vp] * 9 + [_i32] * 6 + [ctypes.c_int, _vp], ctypes.c_int),
     "kda_trace_read": ([ctypes.c_char_p, _i32, ctypes.POINTER(ctypes.c_float), _i32], _i32),
 }
 

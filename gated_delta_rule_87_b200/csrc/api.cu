@@ -109,6 +109,8 @@ kda_status_t run_prefill(gdr::PrefillArgs &a, cudaStream_t s) {
 
 namespace gdr {
 
+void set_last_error(const char *msg) { g_last_error = msg; }
+
 __global__ void check_cu_seqlens_kernel(const int32_t *__restrict__ cu, int num_seqs, int T,
                                         int32_t *status) {
   bool bad = false;

@@ -23,6 +23,9 @@ class TraceScope {
   void *stop_ = nullptr;
 };
 
+// Sets the text kda_last_error() returns on the calling host thread.
+void set_last_error(const char *msg);
+
 struct DecodeArgs {
   const void *q, *k, *v;
   const float *g, *beta;

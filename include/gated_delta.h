@@ -150,6 +150,35 @@ KDA_API kda_status_t gdn_decode_step(const void *q, const void *k, const void *v
                              int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
                              kda_dtype_t io_dtype, void *stream);
 
+/* --------------------------------------------------------------------------
+ * kda_chunk_fwd for callers that cannot allocate device memory (the pages
+ * have no counterpart: this is a deployment convenience).  Some hosts own all
+ * device memory through their own pool and do not let a library call
+ * cudaMalloc, or run where an allocation (which may synchronise the device)
+ * is not allowed.  This call takes the same arguments as kda_chunk_fwd minus
+ * the workspace and runs the same kernels with their scratch in a fixed
+ * 64 MiB array inside this library's device memory; it allocates nothing.
+ *
+ *  - Problems whose kda_chunk_fwd_workspace_size() exceeds 64 MiB are
+ *    rejected with KDA_ERR_WORKSPACE (kda_last_error() gives the sizes);
+ *    use kda_chunk_fwd with a workspace for them.
+ *  - Every device that loads the library keeps the 64 MiB until exit.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress) with that device current; make that first call
+ *    before capturing the stream into a CUDA graph.
+ *  - All calls on a device share the array and it keeps the last call's
+ *    contents (each call resets its own status word).  Calls whose kernels
+ *    overlap on the GPU (different streams or threads) race on it: order
+ *    them on one stream.  A device-side error (an invalid cu_seqlens) leaves
+ *    o and final_state unwritten; this call offers no status word to read.
+ * ------------------------------------------------------------------------ */
+KDA_API kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, const void *v,
+                                           const float *g, const float *beta, void *o,
+                                           const float *initial_state, float *final_state,
+                                           const int32_t *cu_seqlens, int32_t num_seqs,
+                                           int32_t B, int32_t T, int32_t H, int32_t d_k,
+                                           int32_t d_v, kda_dtype_t io_dtype, void *stream);
+
 /* Wait for `stream`, then read the device status word of a prefill workspace.
  * Returns KDA_OK or KDA_ERR_DEVICE_CHECK (device code in *device_code when
  * non-NULL), or KDA_ERR_CUDA.  Synchronises the stream. */

@@ -1,0 +1,64 @@
+"""kda_chunk_fwd_noalloc: the prefill for callers that cannot allocate device
+memory (a host that owns all device memory in its own pool, or a path where
+a cudaMalloc is not allowed).  It keeps its scratch in a fixed 64 MiB array
+inside the library, so it takes no workspace argument.
+
+Checked through the C ABI against kda_chunk_fwd (the entry point with a
+caller workspace) on two calls in a row with different inputs, since the
+shared scratch keeps the previous call's contents.  This file is collected
+last so a stop at the first failure has run every other test first."""
+import ctypes
+
+import numpy as np
+import pytest
+
+from gated_delta_rule_87_b200 import workloads as W
+from parity import TOL_BF16, prefill_device_inputs, rel_l2, to_host
+
+pytestmark = pytest.mark.gpu
+
+
+def _call_noalloc(d, B, T, H, stream):
+    import torch
+    import gated_delta_rule_87_b200 as gdr
+    L = gdr.lib()
+    o = torch.full((B, T, H, 128), float("nan"), dtype=torch.bfloat16, device="cuda")
+    sT = torch.full((B, H, 128, 128), float("nan"), dtype=torch.float32, device="cuda")
+    ptr = lambda t: None if t is None else t.data_ptr()
+    st = L.kda_chunk_fwd_noalloc(ptr(d["q"]), ptr(d["k"]), ptr(d["v"]), ptr(d["g"]),
+                                 ptr(d["beta"]), ptr(o), ptr(d["initial_state"]), ptr(sT),
+                                 None, 0, B, T, H, 128, 128, 1, stream)
+    return st, o, sT
+
+
+def test_noalloc_matches_workspace_entry_point_twice():
+    import torch
+    import gated_delta_rule_87_b200 as gdr
+    stream = torch.cuda.current_stream().cuda_stream
+    results = []
+    for seed, T in ((21, 300), (22, 197)):   # two calls in a row, different shapes and data
+        w = W.WORKLOADS["kda_prefill"].replace(T=T, H_qk=4, H_v=4)
+        x = W.make_prefill(w, seed=seed)
+        d = prefill_device_inputs(x)
+        st, o, sT = _call_noalloc(d, 1, T, 4, stream)
+        assert st == gdr.KDA_OK, gdr.lib().kda_last_error()
+        ro, rs, _ = gdr.kda_chunk_fwd(d["q"], d["k"], d["v"], d["g"], d["beta"],
+                                      d["initial_state"])
+        torch.cuda.synchronize()
+        eo = rel_l2(to_host(o), to_host(ro))
+        es = rel_l2(sT.cpu().numpy(), rs.cpu().numpy())
+        assert np.isfinite(to_host(o)).all()
+        assert eo <= TOL_BF16 and es <= TOL_BF16, (eo, es)
+        results.append((eo, es))
+
+
+def test_noalloc_rejects_problems_beyond_its_scratch():
+    import torch
+    import gated_delta_rule_87_b200 as gdr
+    L = gdr.lib()
+    # T = 4096, H = 32 needs about 200 MB of scratch: far above 64 MiB.
+    fake = 1 << 16  # never dereferenced: the size check comes first
+    st = L.kda_chunk_fwd_noalloc(fake, fake, fake, fake, fake, fake * 2, None, None, None, 0,
+                                 1, 4096, 32, 128, 128, 1, None)
+    assert st == gdr.KDA_ERR_WORKSPACE
+    assert b"64" in L.kda_last_error() or b"67108864" in L.kda_last_error()
