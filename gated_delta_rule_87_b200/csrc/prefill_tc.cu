@@ -54,8 +54,6 @@ using namespace tc;
 
 constexpr int C = kChunk;  // 64 tokens
 constexpr int DK = 128;
-constexpr int NS = 32;  // scan: state columns per CTA
-constexpr int NSL = DK / NS;
 
 // ---- workspace: header, per-sequence chunk offsets, chunk table, slots ----
 struct ChunkEntry {
@@ -64,8 +62,8 @@ struct ChunkEntry {
 constexpr size_t kHeaderBytes = 256;  // [0] status word, [1] number of chunks
 constexpr uint32_t SLOT_P = 0;        // 32 KB  P, K-major A image [i][c]
 constexpr uint32_t SLOT_QP = 32768;   // 16 KB  Q', MN-major A image [c][t]
-constexpr uint32_t SLOT_QC = 49152;   // 32 KB  Qc, bf16 [slice][i][n mod 32]
-constexpr uint32_t SLOT_OI = 81920;   // 16 KB  O_intra, bf16 [slice][t][n mod 32]
+constexpr uint32_t SLOT_QC = 49152;   // 32 KB  Qc^T, bf16 row-major [j][i] (rowimg_off)
+constexpr uint32_t SLOT_OI = 81920;   // 16 KB  O_intra^T, bf16 row-major [j][t] (rowimg_off)
 constexpr uint32_t SLOT_BYTES = 98304;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
@@ -168,18 +166,21 @@ plan_kernel(const int32_t *__restrict__ cu, int num_seqs, int T, int T_total, in
 constexpr int kPrepThreads = 256;
 
 // shared memory map (bytes from a 1024-aligned base)
-constexpr uint32_t OFF_Q = 0;         // q tile, two K-major SW128 [64 t][64 c] blocks
-constexpr uint32_t OFF_K = 16384;     // k tile
+constexpr uint32_t OFF_Q = 0;         // q tile, two K-major SW128 [64 t][64 c] blocks; later q.e^{G}
+constexpr uint32_t OFF_K = 16384;     // k tile; later K.e^{Gp} (same bytes: MN-major [t][c])
 constexpr uint32_t OFF_V = 32768;     // v tile (MN-major operand, 64-wide blocks 8 KB apart)
-constexpr uint32_t OFF_G = 49152;     // g / G fp32 [64][128]
+constexpr uint32_t OFF_G = 49152;     // g fp32 [64][128]; later beta K.e^{G_L-G} | beta K.e^{G_L-Gp}
 constexpr uint32_t OFF_X = 81920;     // 112 KB phase-dependent region
 constexpr uint32_t OFF_MISC = 196608;
 constexpr uint32_t MISC_BETA = 0;      // f32[64]
-constexpr uint32_t MISC_E = 256;       // f32[4][128] sub-chunk-end G
-constexpr uint32_t MISC_GSC = 2304;    // f32[64] scalar gate
-constexpr uint32_t MISC_BAR = 2560;    // 2 x u64
-constexpr uint32_t MISC_TSLOT = 2576;  // u32
-constexpr uint32_t PREP_SMEM = OFF_MISC + 3072 + 1024;
+constexpr uint32_t MISC_GSC = 256;     // f32[64] scalar gate
+constexpr uint32_t MISC_PBLK = 512;    // f32[4][128] product of a over each sub-chunk
+constexpr uint32_t MISC_GSUM = 2560;   // f32[4][128] sum of g over each sub-chunk
+constexpr uint32_t MISC_GLE = 4608;    // f32[128] e^{G_L}
+constexpr uint32_t MISC_BAR = 5120;    // 2 x u64
+constexpr uint32_t MISC_TSLOT = 5136;  // u32
+constexpr uint32_t PREP_SMEM = OFF_MISC + 6144 + 1024;
+constexpr uint32_t OFF_KAB = OFF_G, OFF_KBB = OFF_G + 16384;
 
 // X region, gram phase
 constexpr uint32_t X_R = 0;           // 32 KB, K-major B [128 rows][128], blocks 16 KB apart
@@ -192,15 +193,15 @@ __device__ __forceinline__ uint32_t left_off(int J) {
 constexpr uint32_t X_AWBW = 0;        // 16 KB K-major B [128 i'][64 j]
 constexpr uint32_t X_BE = 16384;      // 8 KB  K-major B [64 i][64 j]
 constexpr uint32_t X_TINVB = 24576;   // 8 KB  K-major B [64 i][64 j]; scratch before
-constexpr uint32_t X_NAE = 32768;     // 16 KB f32 [64][64]
-constexpr uint32_t X_TINVF = 49152;   // 16 KB f32 [64][64]
-constexpr uint32_t X_KP = 65536;      // 16 KB MN-major [t][c]
-constexpr uint32_t X_KAB = 81920;     // 16 KB MN-major [t][i]
-constexpr uint32_t X_KBB = 98304;     // 16 KB MN-major [t][i]
+constexpr int LDN = 68;               // padded row stride (floats) of the fp32 64x64 tiles
+constexpr uint32_t X_NAE = 32768;     // 17 KB f32 [64][LDN]  (N = tril(A_e) diag(beta))
+constexpr uint32_t X_TINVF = 50176;   // 17 KB f32 [64][LDN]  (T^{-1}); both dead after step 6
 constexpr uint32_t X_W = 32768;       // after T2: K-major [c][t]
 constexpr uint32_t X_Y = 49152;       // after T2: K-major [n][t]
 constexpr uint32_t X_U = 65536;       // after T3: K-major [n][t]
-constexpr uint32_t X_OST = 0;         // after T4: bf16 [64 t][128 n]
+constexpr uint32_t X_QPI = 0;         // after T3: Q' image (16 KB), bulk-copied to the slot
+constexpr uint32_t X_PI = 81920;      // after T3: P image (32 KB); after T4: Qc image
+constexpr uint32_t X_OII = 0;         // after T4: O_intra image (16 KB)
 
 // TMEM columns
 constexpr uint32_t TM_GRAM = 0, TM_P = 0, TM_W = 128, TM_QC = 128, TM_YB = 192, TM_OI = 256,
@@ -210,15 +211,11 @@ __device__ __forceinline__ float ld_bf16(const unsigned char *base, uint32_t off
   return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(base + off));
 }
 
-// 8 consecutive bf16 of a K-major SW128 tile row (c multiple of 8)
-__device__ __forceinline__ void ld8_kmajor(const unsigned char *tile, int r, int c, float (&x)[8]) {
-  const uint4 u = *reinterpret_cast<const uint4 *>(tile + (c >> 6) * 8192 + kmajor_off(r, c & 63));
-  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    x[2 * i] = bf16_lo(w[i]);
-    x[2 * i + 1] = bf16_hi(w[i]);
-  }
+// Row-major bf16 images read one row per thread (Qc^T, O_intra^T): the 16-byte
+// chunks of row j are XOR-swizzled by j mod 8 so that 32 threads reading 32
+// rows hit all banks.  Byte offset of chunk `ch` (8 elements) of row j:
+__device__ __forceinline__ uint32_t rowimg_off(int j, int row_bytes, int ch) {
+  return (uint32_t)(j * row_bytes + (((ch & ~7) | ((ch ^ j) & 7)) * 16));
 }
 
 __device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
@@ -242,8 +239,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   float *sG = reinterpret_cast<float *>(sm + OFF_G);
   unsigned char *sX = sm + OFF_X;
   float *sBeta = reinterpret_cast<float *>(sm + OFF_MISC + MISC_BETA);
-  float *sE = reinterpret_cast<float *>(sm + OFF_MISC + MISC_E);
   float *sGsc = reinterpret_cast<float *>(sm + OFF_MISC + MISC_GSC);
+  float *sPblk = reinterpret_cast<float *>(sm + OFF_MISC + MISC_PBLK);
+  float *sGsum = reinterpret_cast<float *>(sm + OFF_MISC + MISC_GSUM);
+  float *sGLe = reinterpret_cast<float *>(sm + OFF_MISC + MISC_GLE);
   uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + OFF_MISC + MISC_BAR);
   uint64_t *bar_mma = bar_tma + 1;
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + MISC_TSLOT);
@@ -290,65 +289,130 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   mbar_wait(bar_tma, 0, hdr, KDA_DEVICE_TIMEOUT);
   __syncthreads();
 
-  // ---- 2. in-chunk cumulative log-decay, rows >= L carry no decay ----
-  if (tid < DK) {
-    const int c = tid;
-    float acc = 0.f;
-    for (int t = 0; t < C; ++t) {
-      const float gv = (t < L) ? (CHANNEL ? sG[t * DK + c] : sGsc[t]) : 0.f;
-      acc += gv;
-      sG[t * DK + c] = acc;
-      if ((t & 15) == 15) sE[(t >> 4) * DK + c] = acc;
+  // ---- 2. per-token decays a = e^{g} (rows >= L: no decay), sub-chunk sums ----
+  // Thread (I, p) owns channels c = 2p, 2p+1 of the 16 tokens of sub-chunk I.
+  // Every in-chunk factor is a product of these a's: with G the in-chunk
+  // cumulative log-decay and E_I its value at the end of sub-chunk I,
+  //   e^{G_t - E_{I-1}} = prefix product of a in sub-chunk I up to t   (<= 1)
+  //   e^{E_I - G_t}     = suffix product after t                       (<= 1)
+  // and factors across sub-chunks are products of whole-sub-chunk products.
+  const int bI = tid >> 6, c2 = (tid & 63) * 2;
+  float a0[16], a1[16];
+  {
+    float s0 = 0.f, s1 = 0.f, p0 = 1.f, p1 = 1.f;
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      const int t = 16 * bI + r;
+      float g0 = 0.f, g1 = 0.f;
+      if (t < L) {
+        if (CHANNEL) {
+          const float2 gg = *reinterpret_cast<const float2 *>(sG + t * DK + c2);
+          g0 = gg.x;
+          g1 = gg.y;
+        } else {
+          g0 = g1 = sGsc[t];
+        }
+      }
+      a0[r] = expf(g0);
+      a1[r] = expf(g1);
+      s0 += g0;
+      s1 += g1;
+      p0 *= a0[r];
+      p1 *= a1[r];
     }
+    sPblk[bI * DK + c2] = p0;
+    sPblk[bI * DK + c2 + 1] = p1;
+    sGsum[bI * DK + c2] = s0;
+    sGsum[bI * DK + c2 + 1] = s1;
   }
-  __syncthreads();
+  __syncthreads();  // g is consumed: its region is reused below
 
-  // ---- 3. Gram operands: R (keys scaled to their sub-chunk end), Left^(J) ----
-  // R row rho = 32J + s: s < 16 -> k_j e^{E_J - G_j}, s >= 16 -> k_j e^{E_J - Gp_j}, j = 16J + s%16
-  for (int item = tid; item < 128 * 16; item += kPrepThreads) {
-    const int rho = item >> 4, c = (item & 15) * 8;
-    const int J = rho >> 5, s = rho & 31, j = 16 * J + (s & 15);
-    float x[8];
-    if (j < L) {
-      ld8_kmajor(sK, j, c, x);
+  // ---- 3. one pass builds every operand of the chunk ----
+  {
+    float F0[4], F1[4];  // e^{E_{I-1} - E_J}: J < I products (<= 1), J = I e^{-sum g} (>= 1)
+    float ei0 = 1.f, ei1 = 1.f, ge0 = 1.f, ge1 = 1.f;  // e^{E_{I-1}}, e^{G_L - E_I}
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float gj = (s < 16) ? sG[j * DK + c + e] : (j > 0 ? sG[(j - 1) * DK + c + e] : 0.f);
-        x[e] *= expf(sE[J * DK + c + e] - gj);
+    for (int J = 0; J < 4; ++J) {
+      if (J < bI) {
+        ei0 *= sPblk[J * DK + c2];
+        ei1 *= sPblk[J * DK + c2 + 1];
       }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = 0.f;
-    }
-    st16(sX + X_R + (c >> 6) * 16384 + kmajor_off(rho, c & 63), pack8(x));
-  }
-  // Left^(J) row lambda = 32I + s (I >= J): s < 16 -> k_i e^{Gp_i - E_J} (i = 16I + s),
-  //                                         s >= 16 -> q_i e^{G_i - E_J} (i = 16I + s - 16)
-  for (int item = tid; item < 320 * 16; item += kPrepThreads) {
-    int r = item >> 4;
-    const int c = (item & 15) * 8;
-    int J = 0;
-    while (r >= 128 - 32 * J) {
-      r -= 128 - 32 * J;
-      ++J;
-    }
-    const int lambda = 32 * J + r;
-    const int I = lambda >> 5, s = lambda & 31;
-    const bool isK = s < 16;
-    const int i = 16 * I + (s & 15);
-    float x[8];
-    if (i < L) {
-      ld8_kmajor(isK ? sK : sQ, i, c, x);
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float gi = isK ? (i > 0 ? sG[(i - 1) * DK + c + e] : 0.f) : sG[i * DK + c + e];
-        x[e] *= expf(gi - sE[J * DK + c + e]);
+      if (J > bI) {
+        ge0 *= sPblk[J * DK + c2];
+        ge1 *= sPblk[J * DK + c2 + 1];
       }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) x[e] = 0.f;
     }
-    st16(sX + X_LEFT + left_off(J) + (c >> 6) * LEFT_BLOCK + kmajor_off(lambda, c & 63), pack8(x));
+#pragma unroll
+    for (int J = 0; J < 4; ++J) {
+      float f0 = 1.f, f1 = 1.f;
+      if (J < bI) {
+#pragma unroll
+        for (int J2 = 0; J2 < 4; ++J2)
+          if (J2 > J && J2 < bI) {
+            f0 *= sPblk[J2 * DK + c2];
+            f1 *= sPblk[J2 * DK + c2 + 1];
+          }
+      } else if (J == bI) {
+        f0 = expf(-sGsum[bI * DK + c2]);
+        f1 = expf(-sGsum[bI * DK + c2 + 1]);
+      }
+      F0[J] = f0;
+      F1[J] = f1;
+    }
+    if (bI == 0) {
+      sGLe[c2] = ge0 * sPblk[c2];  // e^{G_L}: product over all four sub-chunks
+      sGLe[c2 + 1] = ge1 * sPblk[c2 + 1];
+    }
+    // suffix products e^{E_I - G_t}
+    float w0[16], w1[16];
+    w0[15] = 1.f;
+    w1[15] = 1.f;
+#pragma unroll
+    for (int r = 14; r >= 0; --r) {
+      w0[r] = w0[r + 1] * a0[r + 1];
+      w1[r] = w1[r + 1] * a1[r + 1];
+    }
+    float pq0 = 1.f, pq1 = 1.f;  // prefix product through t-1: e^{Gp_t - E_{I-1}}
+#pragma unroll
+    for (int r = 0; r < 16; ++r) {
+      const int t = 16 * bI + r;
+      const uint32_t koff = (c2 >> 6) * 8192 + kmajor_off(t, c2 & 63);
+      const uint32_t kraw = *reinterpret_cast<const uint32_t *>(sK + koff);
+      const uint32_t qraw = *reinterpret_cast<const uint32_t *>(sQ + koff);
+      const bool ok = t < L;
+      const float k0 = ok ? bf16_lo(kraw) : 0.f, k1 = ok ? bf16_hi(kraw) : 0.f;
+      const float q0 = ok ? bf16_lo(qraw) : 0.f, q1 = ok ? bf16_hi(qraw) : 0.f;
+      const float b = sBeta[t];
+      const float bk0 = pq0, bk1 = pq1;                       // e^{Gp_t - E_{I-1}}
+      const float bq0 = pq0 * a0[r], bq1 = pq1 * a1[r];       // e^{G_t - E_{I-1}}
+      const float rw0 = w0[r], rw1 = w1[r];                   // e^{E_I - G_t}
+      const float re0 = rw0 * a0[r], re1 = rw1 * a1[r];       // e^{E_I - Gp_t}
+      pq0 = bq0;
+      pq1 = bq1;
+      const int rowK = 32 * bI + r, rowQ = rowK + 16;
+      // Gram right operand (keys scaled to their sub-chunk end)
+      const uint32_t rb = X_R + (c2 >> 6) * 16384;
+      *reinterpret_cast<uint32_t *>(sX + rb + kmajor_off(rowK, c2 & 63)) = pack_bf16x2(k0 * rw0, k1 * rw1);
+      *reinterpret_cast<uint32_t *>(sX + rb + kmajor_off(rowQ, c2 & 63)) = pack_bf16x2(k0 * re0, k1 * re1);
+      // Gram left operands, one per key sub-chunk J <= I
+#pragma unroll
+      for (int J = 0; J < 4; ++J) {
+        if (J <= bI) {
+          const uint32_t lb = X_LEFT + left_off(J) + (c2 >> 6) * LEFT_BLOCK;
+          *reinterpret_cast<uint32_t *>(sX + lb + kmajor_off(rowK, c2 & 63)) =
+              pack_bf16x2(k0 * bk0 * F0[J], k1 * bk1 * F1[J]);
+          *reinterpret_cast<uint32_t *>(sX + lb + kmajor_off(rowQ, c2 & 63)) =
+              pack_bf16x2(q0 * bq0 * F0[J], q1 * bq1 * F1[J]);
+        }
+      }
+      // K e^{Gp} over k, q e^{G} over q (same element, same owner), beta K e^{G_L - G|Gp}
+      *reinterpret_cast<uint32_t *>(sK + koff) = pack_bf16x2(k0 * bk0 * ei0, k1 * bk1 * ei1);
+      *reinterpret_cast<uint32_t *>(sQ + koff) = pack_bf16x2(q0 * bq0 * ei0, q1 * bq1 * ei1);
+      *reinterpret_cast<uint32_t *>(sm + OFF_KAB + koff) =
+          pack_bf16x2(b * k0 * rw0 * ge0, b * k1 * rw1 * ge1);
+      *reinterpret_cast<uint32_t *>(sm + OFF_KBB + koff) =
+          pack_bf16x2(b * k0 * re0 * ge0, b * k1 * re1 * ge1);
+    }
   }
   fence_async_smem();
   tc_fence_before();
@@ -407,7 +471,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       if (isK) {
 #pragma unroll
         for (int u = 0; u < 16; u += 4)
-          *reinterpret_cast<float4 *>(nae + i * 64 + 16 * J + u) =
+          *reinterpret_cast<float4 *>(nae + i * LDN + 16 * J + u) =
               make_float4(e[u], e[u + 1], e[u + 2], e[u + 3]);
       } else {
 #pragma unroll
@@ -420,77 +484,94 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
     }
   }
-  // K . e^{Gp}, beta K . e^{G_L - G}, beta K . e^{G_L - Gp}  (MN-major [t][c])
-  for (int item = tid; item < 64 * 16; item += kPrepThreads) {
-    const int t = item >> 4, c = (item & 15) * 8;
-    float kp[8], ka[8], kb[8];
-    if (t < L) {
-      float kx[8];
-      ld8_kmajor(sK, t, c, kx);
-      const float b = sBeta[t];
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float G = sG[t * DK + c + e];
-        const float Gp = t > 0 ? sG[(t - 1) * DK + c + e] : 0.f;
-        const float GL = sE[3 * DK + c + e];
-        kp[e] = kx[e] * expf(Gp);
-        ka[e] = b * kx[e] * expf(GL - G);
-        kb[e] = b * kx[e] * expf(GL - Gp);
-      }
-    } else {
-#pragma unroll
-      for (int e = 0; e < 8; ++e) kp[e] = ka[e] = kb[e] = 0.f;
-    }
-    const uint32_t off = mnmajor_off(t, c, 8192);
-    st16(sX + X_KP + off, pack8(kp));
-    st16(sX + X_KAB + off, pack8(ka));
-    st16(sX + X_KBB + off, pack8(kb));
-  }
   __syncthreads();
 
   // ---- 6. T^{-1}, T = I + N, N = tril_{-1}(A_e) diag(beta) (blocked, fp32) ----
   {
     const float *nae = reinterpret_cast<const float *>(sX + X_NAE);
     float *tinv = reinterpret_cast<float *>(sX + X_TINVF);
-    float *tmp = reinterpret_cast<float *>(sX + X_TINVB);  // 16 x 64 f32 scratch
-    if (tid < 64) {  // diagonal 16x16 blocks, one column per thread
-      const int I = tid >> 4, cc = tid & 15;
-      float x[16];
+    float *tmp = reinterpret_cast<float *>(sX + X_TINVB);  // 32 x 32 f32 scratch
+    // (a) the four 16x16 diagonal blocks, one warp each: column sweep
+    //     X = I;  for j: X[r][:] -= N[r][j] X[j][:]  (r > j); lane owns row
+    //     lane/2, columns 8*(lane&1) .. +8, row j is broadcast by shuffles.
+    if (warp < 4) {
+      const int B0 = 16 * warp, r = lane >> 1, c0 = 8 * (lane & 1);
+      float x[8];
 #pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        float acc = (r == cc) ? 1.f : 0.f;
+      for (int u = 0; u < 8; ++u) x[u] = (r == c0 + u) ? 1.f : 0.f;
+      float nrow[16];
 #pragma unroll
-        for (int s2 = 0; s2 < r; ++s2)
-          if (s2 >= cc) acc = fmaf(-nae[(16 * I + r) * 64 + 16 * I + s2], x[s2], acc);
-        x[r] = (r >= cc) ? acc : 0.f;
+      for (int j = 0; j < 16; ++j) nrow[j] = nae[(B0 + r) * LDN + B0 + j];
+#pragma unroll
+      for (int j = 0; j < 15; ++j) {
+        const float m = (r > j) ? nrow[j] : 0.f;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const float xj = __shfl_sync(0xffffffffu, x[u], 2 * j + (lane & 1));
+          x[u] = fmaf(-m, xj, x[u]);
+        }
       }
 #pragma unroll
-      for (int r = 0; r < 16; ++r) {
-        tinv[(16 * I + r) * 64 + 16 * I + cc] = x[r];
-#pragma unroll
-        for (int J = 0; J < 4; ++J)
-          if (J > I) tinv[(16 * I + r) * 64 + 16 * J + cc] = 0.f;
-      }
+      for (int u = 0; u < 8; ++u) tinv[(B0 + r) * LDN + B0 + c0 + u] = x[u];
+    }
+    // zero the strictly upper blocks
+    for (int e = tid; e < 64 * 64; e += kPrepThreads) {
+      const int rr = e >> 6, cc = e & 63;
+      if ((cc >> 4) > (rr >> 4)) tinv[rr * LDN + cc] = 0.f;
     }
     __syncthreads();
-    const int r = tid >> 4, cc = tid & 15;
-    for (int I = 1; I < 4; ++I) {
-      for (int J = 0; J < I; ++J) {
-        float acc = 0.f;
-        for (int K2 = J; K2 < I; ++K2)
+    // (b) 32x32 level: T^{-1}[2p+1][2p] = -T^{-1}[2p+1][2p+1] N[2p+1][2p] T^{-1}[2p][2p]
+    {
+      const int pp = tid >> 7, r = (tid >> 3) & 15, cq = (tid & 7) * 2;
+      const int R0 = 32 * pp + 16, C0 = 32 * pp;  // block row / column offsets
+      float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll
-          for (int s2 = 0; s2 < 16; ++s2)
-            acc = fmaf(nae[(16 * I + r) * 64 + 16 * K2 + s2], tinv[(16 * K2 + s2) * 64 + 16 * J + cc], acc);
-        tmp[r * 64 + 16 * J + cc] = acc;
+      for (int s2 = 0; s2 < 16; ++s2) {
+        const float nv = nae[(R0 + r) * LDN + C0 + s2];
+        acc0 = fmaf(nv, tinv[(C0 + s2) * LDN + C0 + cq], acc0);
+        acc1 = fmaf(nv, tinv[(C0 + s2) * LDN + C0 + cq + 1], acc1);
       }
+      tmp[(16 * pp + r) * 32 + cq] = acc0;
+      tmp[(16 * pp + r) * 32 + cq + 1] = acc1;
       __syncthreads();
-      for (int J = 0; J < I; ++J) {
-        float acc = 0.f;
+      acc0 = acc1 = 0.f;
 #pragma unroll
-        for (int s2 = 0; s2 < 16; ++s2)
-          acc = fmaf(tinv[(16 * I + r) * 64 + 16 * I + s2], tmp[s2 * 64 + 16 * J + cc], acc);
-        tinv[(16 * I + r) * 64 + 16 * J + cc] = -acc;
+      for (int s2 = 0; s2 < 16; ++s2) {
+        const float tv = tinv[(R0 + r) * LDN + R0 + s2];
+        acc0 = fmaf(tv, tmp[(16 * pp + s2) * 32 + cq], acc0);
+        acc1 = fmaf(tv, tmp[(16 * pp + s2) * 32 + cq + 1], acc1);
       }
+      tinv[(R0 + r) * LDN + C0 + cq] = -acc0;
+      tinv[(R0 + r) * LDN + C0 + cq + 1] = -acc1;
+      __syncthreads();
+    }
+    // (c) 64x64 level: T^{-1}[lo][hi] = -T^{-1}[lo][lo] N[lo][hi] T^{-1}[hi][hi] (32x32 blocks)
+    {
+      const int r = tid >> 3, cq = (tid & 7) * 4;
+      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+      for (int s2 = 0; s2 < 32; ++s2) {
+        const float nv = nae[(32 + r) * LDN + s2];
+        const float4 tv = *reinterpret_cast<const float4 *>(tinv + s2 * LDN + cq);
+        acc[0] = fmaf(nv, tv.x, acc[0]);
+        acc[1] = fmaf(nv, tv.y, acc[1]);
+        acc[2] = fmaf(nv, tv.z, acc[2]);
+        acc[3] = fmaf(nv, tv.w, acc[3]);
+      }
+      *reinterpret_cast<float4 *>(tmp + r * 32 + cq) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      __syncthreads();
+      acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+#pragma unroll 8
+      for (int s2 = 0; s2 < 32; ++s2) {
+        const float tv = tinv[(32 + r) * LDN + 32 + s2];
+        const float4 xv = *reinterpret_cast<const float4 *>(tmp + s2 * 32 + cq);
+        acc[0] = fmaf(tv, xv.x, acc[0]);
+        acc[1] = fmaf(tv, xv.y, acc[1]);
+        acc[2] = fmaf(tv, xv.z, acc[2]);
+        acc[3] = fmaf(tv, xv.w, acc[3]);
+      }
+      *reinterpret_cast<float4 *>(tinv + (32 + r) * LDN + cq) =
+          make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
       __syncthreads();
     }
     // bf16 copy, K-major [i][j]
@@ -498,7 +579,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const int i = item >> 3, j = (item & 7) * 8;
       float x[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = tinv[i * 64 + j + u];
+      for (int u = 0; u < 8; ++u) x[u] = tinv[i * LDN + j + u];
       st16(sX + X_TINVB + kmajor_off(i, j), pack8(x));
     }
   }
@@ -512,7 +593,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t tinvb = smem_u32(sX + X_TINVB);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_W, desc_mnmajor(smem_u32(sX + X_KP), 16 * kk, 8192),
+      mma_bf16(tm + TM_W, desc_mnmajor(smem_u32(sK), 16 * kk, 8192),
                desc_kmajor(tinvb, 16 * kk, 0), idesc_bf16(128, 64, true, false), kk > 0);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
@@ -561,7 +642,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                idesc_bf16(128, 64, false, false), kk > 0);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_P, desc_mnmajor(smem_u32(sX + X_KBB), 16 * kk, 8192), desc_kmajor(wsm, 16 * kk, 0),
+      mma_bf16(tm + TM_P, desc_mnmajor(smem_u32(sm + OFF_KBB), 16 * kk, 8192), desc_kmajor(wsm, 16 * kk, 0),
                idesc_bf16(128, 128, true, false), kk > 0);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
@@ -585,9 +666,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       for (int u = 0; u < 8; ++u) x[u] = v[8 * seg + u];
       st16(sX + X_U + kmajor_off(lane_row, 32 * half + 8 * seg), pack8(x));
     }
-    // P = Diag(e^{G_L}) - K_b^T beta W (lanes i, cols c) -> slot, K-major A image
+    // P = Diag(e^{G_L}) - K_b^T beta W (lanes i, cols c) -> K-major A image [i][c]
     const int i = lane_row;
-    const float gl = expf(sE[3 * DK + i]);
+    const float gl = sGLe[i];
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
       const int c0 = 64 * half + 32 * part;
@@ -602,10 +683,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           x[u] = (c == i ? gl : 0.f) - v[8 * seg + u];
         }
         const int c = c0 + 8 * seg;
-        st16(slot + SLOT_P + (c >> 6) * 16384 + kmajor_off(i, c & 63), pack8(x));
+        st16(sX + X_PI + (c >> 6) * 16384 + kmajor_off(i, c & 63), pack8(x));
       }
     }
-    // Q'[t][c] = q_tc e^{G_tc} - X[c][t] (lanes c, cols t) -> slot, MN-major A image [c][t]
+    // Q'[t][c] = q_tc e^{G_tc} - X[c][t] (lanes c, cols t) -> MN-major A image [c][t]
     const int c = lane_row;
     tmem_ld32(taddr(tm, 32 * quad, TM_X + 32 * half), v);
     tmem_ld_wait();
@@ -615,72 +696,84 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int t = 32 * half + 8 * seg + u;
-        const float qv = ld_bf16(sQ, (c >> 6) * 8192 + kmajor_off(t, c & 63));
-        x[u] = (t < L) ? qv * expf(sG[t * DK + c]) - v[8 * seg + u] : 0.f;
+        const float qg = ld_bf16(sQ, (c >> 6) * 8192 + kmajor_off(t, c & 63));  // q e^{G}
+        x[u] = (t < L) ? qg - v[8 * seg + u] : 0.f;
       }
-      st16(slot + SLOT_QP + sw128((uint32_t)(c * 128 + (32 * half + 8 * seg) * 2)), pack8(x));
+      st16(sX + X_QPI + sw128((uint32_t)(c * 128 + (32 * half + 8 * seg) * 2)), pack8(x));
     }
   }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
+  if (tid == 0) {  // P and Q' images -> workspace slot
+    bulk_s2g(slot + SLOT_P, sX + X_PI, 32768);
+    bulk_s2g(slot + SLOT_QP, sX + X_QPI, 16384);
+    bulk_commit();
+  }
 
-  // ---- 9. O_intra^T -= U^T (B_e beta)^T;  Qc = (K_a beta)^T V - (K_b beta)^T U ----
+  // ---- 9. O_intra^T -= U^T (B_e beta)^T;  Qc^T = V^T beta K_a - U^T beta K_b ----
   if (tid == 0) {
     const uint32_t usm = smem_u32(sX + X_U);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_OI, desc_kmajor(usm, 16 * kk, 0), desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0),
                idesc_bf16(128, 64, false, false, true), 1);
+    // Qc^T = V^T (beta K e^{G_L-G}) - U^T (beta K e^{G_L-Gp}): lanes j, columns i
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sX + X_KAB), 16 * kk, 8192),
-               desc_mnmajor(smem_u32(sV), 16 * kk, 8192), idesc_bf16(128, 128, true, true), kk > 0);
+      mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sV), 16 * kk, 8192),
+               desc_mnmajor(smem_u32(sm + OFF_KAB), 16 * kk, 8192), idesc_bf16(128, 128, true, true),
+               kk > 0);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sX + X_KBB), 16 * kk, 8192), desc_kmajor(usm, 16 * kk, 0),
-               idesc_bf16(128, 128, true, false, true), 1);
+      mma_bf16(tm + TM_QC, desc_kmajor(usm, 16 * kk, 0),
+               desc_mnmajor(smem_u32(sm + OFF_KBB), 16 * kk, 8192),
+               idesc_bf16(128, 128, false, true, true), 1);
     mma_commit(bar_mma);
   }
   __syncwarp();
   mbar_wait(bar_mma, 1, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
 
+  if (tid == 0) bulk_wait_read0();  // the P / Q' images may now be overwritten
+  __syncthreads();
   {
     float v[32];
-    // O_intra (lanes n, cols t) -> staging [t][n]
-    const int n = lane_row;
+    // O_intra^T (lanes j, cols t) -> image row-major [j][t]
+    const int j = lane_row;
     tmem_ld32(taddr(tm, 32 * quad, TM_OI + 32 * half), v);
     tmem_ld_wait();
-    __nv_bfloat16 *ost = reinterpret_cast<__nv_bfloat16 *>(sX + X_OST);
 #pragma unroll
-    for (int u = 0; u < 32; ++u) ost[(32 * half + u) * DK + n] = __float2bfloat16_rn(v[u]);
-    // Qc (lanes i, cols n) -> slot [slice][i][n mod 32]
-    const int i = lane_row;
+    for (int seg = 0; seg < 4; ++seg) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = v[8 * seg + u];
+      st16(sX + X_OII + rowimg_off(j, C * 2, 4 * half + seg), pack8(x));
+    }
+    // Qc^T (lanes j, cols i) -> image row-major [j][i]
 #pragma unroll
     for (int part = 0; part < 2; ++part) {
-      const int n0 = 64 * half + 32 * part;  // one 32-wide slice
-      tmem_ld32(taddr(tm, 32 * quad, TM_QC + n0), v);
+      const int i0 = 64 * half + 32 * part;
+      tmem_ld32(taddr(tm, 32 * quad, TM_QC + i0), v);
       tmem_ld_wait();
-      const int sl = n0 / NS;
 #pragma unroll
       for (int seg = 0; seg < 4; ++seg) {
         float x[8];
 #pragma unroll
         for (int u = 0; u < 8; ++u) x[u] = v[8 * seg + u];
-        st16(slot + SLOT_QC + ((sl * DK + i) * NS + 8 * seg) * 2, pack8(x));
+        st16(sX + X_PI + rowimg_off(j, DK * 2, i0 / 8 + seg), pack8(x));
       }
     }
   }
+  fence_async_smem();
   tc_fence_before();
   __syncthreads();
-  // staging -> slot [slice][t][n mod 32]
-  for (int item = tid; item < 64 * 16; item += kPrepThreads) {
-    const int t = item >> 4, n8 = (item & 15) * 8;
-    const uint4 u = *reinterpret_cast<const uint4 *>(sX + X_OST + (t * DK + n8) * 2);
-    const int sl = n8 / NS;
-    *reinterpret_cast<uint4 *>(slot + SLOT_OI + ((sl * C + t) * NS + (n8 % NS)) * 2) = u;
+  if (tid == 0) {
+    bulk_s2g(slot + SLOT_QC, sX + X_PI, 32768);
+    bulk_s2g(slot + SLOT_OI, sX + X_OII, 16384);
+    bulk_commit();
+    bulk_wait0();
   }
   if (warp == 0) tmem_dealloc(tm, 512);
 }
@@ -688,13 +781,32 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 // ---------------------------------------------------------------------------
 // scan kernel
 // ---------------------------------------------------------------------------
-constexpr int kScanThreads = 128;
-constexpr uint32_t ST_P = 0, ST_QP = 32768, ST_QC = 49152, ST_OI = 57344, ST_BYTES = 65536;
-constexpr uint32_t SC_SB = 2 * ST_BYTES;  // 8 KB S operand, K-major [n][i] (two 4 KB blocks)
-constexpr uint32_t SC_MISC = SC_SB + 8192;
-constexpr uint32_t SCAN_SMEM = SC_MISC + 128 + 1024;
-constexpr uint32_t STAGE_TX = 32768 + 16384 + 8192 + 4096;
+constexpr int NSTAGE = 2;
+constexpr uint32_t ST_P = 0, ST_QP = 32768, ST_QC = 49152, ST_OI = 81920, ST_BYTES = 98304;
+constexpr uint32_t SC_OT = NSTAGE * ST_BYTES;  // 16 KB output tile [t][j] bf16
+constexpr uint32_t SC_MISC = SC_OT + 16384;
+constexpr uint32_t SCAN_SMEM = SC_MISC + 256 + 1024;
+constexpr uint32_t STAGE_TX = SLOT_BYTES;
+// TMEM columns: S^T operand (bf16 pairs) x3, D_s = (P S)^T, D_o = (Q' S)^T x2
+constexpr uint32_t TA0 = 0, TD_S = 192, TD_O = 320;
+// warp roles
+constexpr int kChainWarps = 8;   // warps 0-7: state column j = lane quadrant, half of the rows
+constexpr int kOutWarps = 4;     // warps 8-11: outputs
+constexpr int kMmaWarp = 12;
+constexpr int kLoadWarp = 13;
+constexpr int kScanThreads = 32 * 14;
+constexpr int kOutBarrier = 1;   // named barrier among the output warps
 
+// The scan walks one sequence's chunks for one v-head, computing the
+// transposed state S^T (lanes = value column j, d_k along TMEM columns):
+//     (S_{u+1})^T = S_u^T P_u^T + Qc_u^T ,      o_u^T = S_u^T Q'_u^T + O_intra_u^T
+// S_u^T lives in TMEM as the bf16 A operand, so the serial chain is
+//   tcgen05.ld (P S)^T -> + Qc^T -> tcgen05.st bf16 -> 8 MMAs (128x128x16)
+// and never touches shared memory.  Roles, connected by mbarriers:
+//   chain warps  : S^T update, rows [64*half, 64*half + 64) of lane j
+//   MMA warp     : P_u products, then the previous chunk's Q' product
+//   output warps : o_u = (D_o)^T + O_intra -> shared tile -> global
+//   load warp    : chunk inputs into NSTAGE stages (bulk copies)
 __global__ void __launch_bounds__(kScanThreads, 1)
 chunk_scan_kernel(const int32_t *hdr, const int32_t *__restrict__ seq_off,
                   const ChunkEntry *__restrict__ tab, const unsigned char *__restrict__ slots,
@@ -703,137 +815,194 @@ chunk_scan_kernel(const int32_t *hdr, const int32_t *__restrict__ seq_off,
   extern __shared__ unsigned char smem_raw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
-  uint64_t *full = reinterpret_cast<uint64_t *>(sm + SC_MISC);
-  uint64_t *mma_bar = full + 2;
-  uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + SC_MISC + 64);
-  unsigned char *sb = sm + SC_SB;
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + SC_MISC);  // [NSTAGE]
+  uint64_t *empty = full + NSTAGE;                              // [NSTAGE], chain + out arrivals
+  uint64_t *op_ready = empty + NSTAGE;                          // [3], chain arrivals
+  uint64_t *o_free = op_ready + 3;                              // [2], out arrivals
+  uint64_t *bar_s = o_free + 2;                                 // commit
+  uint64_t *bar_o = bar_s + 1;                                  // [2], commit
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + SC_MISC + 192);
 
   if (hdr[0] != KDA_DEVICE_OK) return;
-  const int n = blockIdx.x / NSL, sl = blockIdx.x % NSL, h = blockIdx.y;
+  const int n = blockIdx.x, h = blockIdx.y;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int c_begin = seq_off[n], c_end = seq_off[n + 1];
   const int nch = c_end - c_begin;
 
   if (warp == 0) {
-    tmem_alloc(tslot, 64);
+    tmem_alloc(tslot, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(&full[0], 1);
-    mbar_init(&full[1], 1);
-    mbar_init(mma_bar, 1);
+    for (int st = 0; st < NSTAGE; ++st) {
+      mbar_init(&full[st], 1);
+      mbar_init(&empty[st], 32 * (kChainWarps + kOutWarps));
+    }
+    for (int b = 0; b < 3; ++b) mbar_init(&op_ready[b], 32 * kChainWarps);
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&o_free[b], 32 * kOutWarps);
+      mbar_init(&bar_o[b], 1);
+    }
+    mbar_init(bar_s, 1);
     mbar_fence_init();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tslot;
+  const size_t state_base = ((size_t)n * H_v + h) * DK * DK;
 
-  auto load_stage = [&](int u) {
-    const int st = u & 1;
-    const unsigned char *slot = slots + ((size_t)(c_begin + u) * H_v + h) * SLOT_BYTES;
-    unsigned char *dst = sm + st * ST_BYTES;
-    mbar_arrive_expect_tx(&full[st], STAGE_TX);
-    bulk_g2s(dst + ST_P, slot + SLOT_P, 32768, &full[st]);
-    bulk_g2s(dst + ST_QP, slot + SLOT_QP, 16384, &full[st]);
-    bulk_g2s(dst + ST_QC, slot + SLOT_QC + sl * (DK * NS * 2), DK * NS * 2, &full[st]);
-    bulk_g2s(dst + ST_OI, slot + SLOT_OI + sl * (C * NS * 2), C * NS * 2, &full[st]);
-  };
-  if (tid == 0) {
-    if (nch > 0) load_stage(0);
-    if (nch > 1) load_stage(1);
-  }
-
-  // state row i = tid, columns [sl*32, sl*32 + 32)
-  const int i = tid;
-  float S[NS];
-  const size_t soff = ((size_t)n * H_v + h) * DK * DK + (size_t)i * DK + sl * NS;
+  if (warp == kLoadWarp) {
+    // ---------------- loads ----------------
+    if (lane == 0) {
+      constexpr int kAhead = 4;  // chunks prefetched into L2 ahead of their stage load
+      for (int u = 0; u < kAhead && u < nch; ++u)
+        bulk_prefetch_l2(slots + ((size_t)(c_begin + u) * H_v + h) * SLOT_BYTES, SLOT_BYTES);
+      for (int u = 0; u < nch; ++u) {
+        const int st = u % NSTAGE;
+        if (u + kAhead < nch)
+          bulk_prefetch_l2(slots + ((size_t)(c_begin + u + kAhead) * H_v + h) * SLOT_BYTES,
+                           SLOT_BYTES);
+        if (u >= NSTAGE) mbar_wait(&empty[st], ((u - NSTAGE) / NSTAGE) & 1, err, KDA_DEVICE_TIMEOUT);
+        mbar_arrive_expect_tx(&full[st], STAGE_TX);
+        bulk_g2s(sm + st * ST_BYTES, slots + ((size_t)(c_begin + u) * H_v + h) * SLOT_BYTES,
+                 SLOT_BYTES, &full[st]);
+      }
+    }
+  } else if (warp == kMmaWarp) {
+    // ---------------- tensor-core issue ----------------
+    if (lane == 0) {
+      auto q_product = [&](int u) {  // o_u^T = S_u^T Q'_u^T  (M = 128 j, N = 64 t)
+        const uint32_t qa = smem_u32(sm + (u % NSTAGE) * ST_BYTES + ST_QP);
+        if (u >= 2) mbar_wait(&o_free[u & 1], ((u - 2) >> 1) & 1, err, KDA_DEVICE_TIMEOUT);
+        tc_fence_after();
 #pragma unroll
-  for (int u = 0; u < NS; u += 4) {
-    float4 x = s0 ? *reinterpret_cast<const float4 *>(s0 + soff + u) : make_float4(0.f, 0.f, 0.f, 0.f);
-    S[u] = x.x; S[u + 1] = x.y; S[u + 2] = x.z; S[u + 3] = x.w;
-  }
-
-  for (int u = 0; u < nch; ++u) {
-    const int st = u & 1;
-    const uint32_t ph = (u >> 1) & 1;
-    const unsigned char *stage = sm + st * ST_BYTES;
-    // S (bf16) -> K-major B operand [n][i]
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tm + TD_O + 64 * (u & 1), tm + TA0 + 64 * (u % 3) + 8 * kk,
+                      desc_mnmajor(qa, 16 * kk, 0), idesc_bf16(128, 64, false, true), kk > 0);
+        mma_commit(&bar_o[u & 1]);
+      };
+      for (int u = 0; u < nch; ++u) {
+        const int st = u % NSTAGE;
+        mbar_wait(&op_ready[u % 3], (u / 3) & 1, err, KDA_DEVICE_TIMEOUT);
+        mbar_wait(&full[st], (u / NSTAGE) & 1, err, KDA_DEVICE_TIMEOUT);
+        tc_fence_after();
+        const uint32_t pa = smem_u32(sm + st * ST_BYTES + ST_P);
+        // (P S)^T = S^T P^T  (M = 128 j, N = 128 i, K = 128 c); B = P rows, K-major
 #pragma unroll
-    for (int nn = 0; nn < NS; ++nn)
-      *reinterpret_cast<__nv_bfloat16 *>(sb + (i >> 6) * 4096 + kmajor_off(nn, i & 63)) =
-          __float2bfloat16_rn(S[nn]);
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    tc_fence_after();
-    mbar_wait(&full[st], ph, err, KDA_DEVICE_TIMEOUT);
-    if (tid == 0) {
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16_ts(tm + TD_S, tm + TA0 + 64 * (u % 3) + 8 * kk, desc_kmajor(pa, 16 * kk, 16384),
+                      idesc_bf16(128, 128, false, false), kk > 0);
+        mma_commit(bar_s);
+        q_product(u);  // overlaps the chain's state update
+      }
+    }
+  } else if (warp < kChainWarps) {
+    // ---------------- the state chain: column j, rows [64*hh, 64*hh + 64) ----------------
+    const int q4 = warp & 3, hh = warp >> 2;
+    const int j = 32 * q4 + lane;
+    float S[64];
+#pragma unroll
+    for (int r = 0; r < 64; ++r)
+      S[r] = s0 ? s0[state_base + (size_t)(64 * hh + r) * DK + j] : 0.f;
+    auto write_operand = [&](int buf) {  // S^T rows -> bf16 pairs in TMEM
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(S[2 * c], S[2 * c + 1]);
+      tmem_st32(taddr(tm, 32 * q4, TA0 + 64 * buf + 32 * hh), pk);
+      tmem_st_wait();
+      tc_fence_before();
+    };
+    if (nch > 0) {
+      write_operand(0);
+      mbar_arrive(&op_ready[0]);
+    }
+    for (int u = 0; u < nch; ++u) {
+      const int st = u % NSTAGE;
+      mbar_wait(bar_s, u & 1, err, KDA_DEVICE_TIMEOUT);
       tc_fence_after();
-      const uint32_t pa = smem_u32(stage + ST_P), qa = smem_u32(stage + ST_QP), sbb = smem_u32(sb);
+      float v[32];
+      const unsigned char *qc = sm + st * ST_BYTES + ST_QC;
+      mbar_wait(&full[st], (u / NSTAGE) & 1, err, KDA_DEVICE_TIMEOUT);
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tm, desc_kmajor(pa, 16 * kk, 16384), desc_kmajor(sbb, 16 * kk, 4096),
-                 idesc_bf16(128, NS, false, false), kk > 0);
+      for (int part = 0; part < 2; ++part) {
+        tmem_ld32(taddr(tm, 32 * q4, TD_S + 64 * hh + 32 * part), v);
+        tmem_ld_wait();
 #pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tm + 32, desc_mnmajor(qa, 16 * kk, 0), desc_kmajor(sbb, 16 * kk, 4096),
-                 idesc_bf16(64, NS, true, false), kk > 0);
-      mma_commit(mma_bar);
-    }
-    __syncwarp();
-    mbar_wait(mma_bar, u & 1, err, KDA_DEVICE_TIMEOUT);
-    tc_fence_after();
-
-    // S <- P S + Qc
-    float v[32];
-    tmem_ld32(taddr(tm, 32 * warp, 0), v);
-    tmem_ld_wait();
-    const uint4 *qc = reinterpret_cast<const uint4 *>(stage + ST_QC + i * NS * 2);
+        for (int seg = 0; seg < 4; ++seg) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(
+              qc + rowimg_off(j, DK * 2, 8 * hh + 4 * part + seg));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
-    for (int seg = 0; seg < NS / 8; ++seg) {
-      const uint4 w = qc[seg];
-      const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        S[8 * seg + 2 * e] = v[8 * seg + 2 * e] + bf16_lo(ww[e]);
-        S[8 * seg + 2 * e + 1] = v[8 * seg + 2 * e + 1] + bf16_hi(ww[e]);
-      }
-    }
-    // o = Q' S + O_intra  (M = 64 accumulator: row t in lane 32*(t/16) + t%16)
-    tmem_ld32(taddr(tm, 32 * warp, 32), v);
-    tmem_ld_wait();
-    const ChunkEntry ce = tab[c_begin + u];
-    const int t = 16 * warp + lane;
-    if (lane < 16 && t < ce.len) {
-      const uint4 *oi = reinterpret_cast<const uint4 *>(stage + ST_OI + t * NS * 2);
-      __nv_bfloat16 *dst = o + ((size_t)(ce.start + t) * H_v + h) * DK + sl * NS;
-#pragma unroll
-      for (int seg = 0; seg < NS / 8; ++seg) {
-        const uint4 w = oi[seg];
-        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-        float x[8];
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          x[2 * e] = v[8 * seg + 2 * e] + bf16_lo(ww[e]);
-          x[2 * e + 1] = v[8 * seg + 2 * e + 1] + bf16_hi(ww[e]);
+          for (int e = 0; e < 4; ++e) {
+            S[32 * part + 8 * seg + 2 * e] = v[8 * seg + 2 * e] + bf16_lo(ww[e]);
+            S[32 * part + 8 * seg + 2 * e + 1] = v[8 * seg + 2 * e + 1] + bf16_hi(ww[e]);
+          }
         }
-        *reinterpret_cast<uint4 *>(dst + 8 * seg) = pack8(x);
       }
+      if (u + 1 < nch) {
+        write_operand((u + 1) % 3);
+        mbar_arrive(&op_ready[(u + 1) % 3]);
+      } else {
+        tc_fence_before();
+      }
+      mbar_arrive(&empty[st]);
     }
-    tc_fence_before();
-    __syncthreads();  // stage, TMEM and the S operand are free again
-    if (tid == 0 && u + 2 < nch) load_stage(u + 2);
+    if (sT) {
+#pragma unroll
+      for (int r = 0; r < 64; ++r) sT[state_base + (size_t)(64 * hh + r) * DK + j] = S[r];
+    }
+  } else if (warp < kChainWarps + kOutWarps) {
+    // ---------------- outputs: o = Q' S + O_intra ----------------
+    const int q4 = warp & 3;
+    const int j = 32 * q4 + lane;
+    const int otid = tid - 32 * kChainWarps;  // 0..127
+    __nv_bfloat16 *tile = reinterpret_cast<__nv_bfloat16 *>(sm + SC_OT);
+    ChunkEntry ce = nch > 0 ? tab[c_begin] : ChunkEntry{0, 0, 0, 0};
+    for (int u = 0; u < nch; ++u) {
+      const int st = u % NSTAGE;
+      const ChunkEntry ce_next = (u + 1 < nch) ? tab[c_begin + u + 1] : ce;
+      mbar_wait(&bar_o[u & 1], (u >> 1) & 1, err, KDA_DEVICE_TIMEOUT);
+      tc_fence_after();
+      mbar_wait(&full[st], (u / NSTAGE) & 1, err, KDA_DEVICE_TIMEOUT);
+      const unsigned char *oi = sm + st * ST_BYTES + ST_OI;
+#pragma unroll
+      for (int part = 0; part < 2; ++part) {
+        float v[32];
+        tmem_ld32(taddr(tm, 32 * q4, TD_O + 64 * (u & 1) + 32 * part), v);
+        tmem_ld_wait();
+#pragma unroll
+        for (int seg = 0; seg < 4; ++seg) {
+          const uint4 w =
+              *reinterpret_cast<const uint4 *>(oi + rowimg_off(j, C * 2, 4 * part + seg));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            const int t = 32 * part + 8 * seg + 2 * e;
+            tile[t * DK + j] = __float2bfloat16_rn(v[8 * seg + 2 * e] + bf16_lo(ww[e]));
+            tile[(t + 1) * DK + j] = __float2bfloat16_rn(v[8 * seg + 2 * e + 1] + bf16_hi(ww[e]));
+          }
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(&o_free[u & 1]);
+      mbar_arrive(&empty[st]);
+      asm volatile("bar.sync %0, %1;" ::"n"(kOutBarrier), "n"(32 * kOutWarps) : "memory");
+      // tile rows t < len -> o[(start + t), h, :]  (16-byte stores, 256 B per row)
+      for (int item = otid; item < C * 16; item += 32 * kOutWarps) {
+        const int t = item >> 4, c8 = (item & 15) * 8;
+        if (t < ce.len)
+          *reinterpret_cast<uint4 *>(o + ((size_t)(ce.start + t) * H_v + h) * DK + c8) =
+              *reinterpret_cast<const uint4 *>(tile + t * DK + c8);
+      }
+      asm volatile("bar.sync %0, %1;" ::"n"(kOutBarrier), "n"(32 * kOutWarps) : "memory");
+      ce = ce_next;
+    }
   }
 
-  if (sT) {
-#pragma unroll
-    for (int u = 0; u < NS; u += 4)
-      *reinterpret_cast<float4 *>(sT + soff + u) = make_float4(S[u], S[u + 1], S[u + 2], S[u + 3]);
-  }
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tm, 64);
+  if (warp == 0) tmem_dealloc(tm, 512);
 }
 
 // ---------------------------------------------------------------------------
@@ -925,7 +1094,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
 
   e = cudaFuncSetAttribute(chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM);
   if (e != cudaSuccess) return e;
-  dim3 gs((unsigned)(a.num_seqs * NSL), (unsigned)a.H_v);
+  dim3 gs((unsigned)a.num_seqs, (unsigned)a.H_v);
   {
     TraceScope tr("chunk_scan_kernel", stream);
     chunk_scan_kernel<<<gs, kScanThreads, SCAN_SMEM, stream>>>(
