@@ -163,7 +163,7 @@ plan_kernel(const int32_t *__restrict__ cu, int num_seqs, int T, int T_total, in
 // ---------------------------------------------------------------------------
 // prep kernel
 // ---------------------------------------------------------------------------
-constexpr int kPrepThreads = 256;
+constexpr int kPrepThreads = 512;
 
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_Q = 0;         // q tile, two K-major SW128 [64 t][64 c] blocks; later q.e^{G}
@@ -233,8 +233,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                   int H_v, int32_t *hdr, const ChunkEntry *__restrict__ tab,
                   unsigned char *__restrict__ slots) {
   extern __shared__ unsigned char smem_raw[];
-  unsigned char *sm = reinterpret_cast<unsigned char *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  // 1024-byte aligned base, derived by pointer arithmetic on the shared array so
+  // that the compiler keeps shared-memory addressing for every access
+  unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   unsigned char *sQ = sm + OFF_Q, *sK = sm + OFF_K, *sV = sm + OFF_V;
   float *sG = reinterpret_cast<float *>(sm + OFF_G);
   unsigned char *sX = sm + OFF_X;
@@ -248,14 +249,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + MISC_TSLOT);
 
   if (hdr[0] != KDA_DEVICE_OK) return;
-  const int chunk = blockIdx.x;
-  if (chunk >= hdr[1]) return;
-  const int h = blockIdx.y;
-  const int hk = h / (H_v / H_qk);
-  const ChunkEntry ce = tab[chunk];
-  const int L = ce.len, t0 = ce.start;
+  // persistent: this CTA walks (chunk, v-head) work items blockIdx.x,
+  // blockIdx.x + gridDim.x, ...; the next item's tiles are loaded while the
+  // current one finishes.
+  const int total = hdr[1] * H_v;
+  int work = blockIdx.x;
+  if (work >= total) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  unsigned char *slot = slots + ((size_t)chunk * H_v + h) * SLOT_BYTES;
 
   if (warp == 0) {
     tmem_alloc(tslot, 512);
@@ -271,38 +271,66 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   tc_fence_after();
   const uint32_t tm = *tslot;
 
-  // ---- 1. TMA loads of the chunk's q, k, v (bf16, swizzled) and g (fp32) ----
-  if (tid == 0) {
+  // ---- 1. TMA loads of an item's q, k, v (bf16, swizzled) and g (fp32) ----
+  auto issue_loads = [&](int w) {  // thread 0
+    const int ck = w / H_v, hh = w - ck * H_v, hkk = hh / (H_v / H_qk);
+    const int ts = tab[ck].start;
+    fence_async_smem();
     mbar_arrive_expect_tx(bar_tma, 3 * 16384 + (CHANNEL ? 32768 : 0));
 #pragma unroll
     for (int cb = 0; cb < 2; ++cb) {
-      tma_load_3d(sQ + cb * 8192, &tm_q, cb * 64, hk, t0, bar_tma);
-      tma_load_3d(sK + cb * 8192, &tm_k, cb * 64, hk, t0, bar_tma);
-      tma_load_3d(sV + cb * 8192, &tm_v, cb * 64, h, t0, bar_tma);
+      tma_load_3d(sQ + cb * 8192, &tm_q, cb * 64, hkk, ts, bar_tma);
+      tma_load_3d(sK + cb * 8192, &tm_k, cb * 64, hkk, ts, bar_tma);
+      tma_load_3d(sV + cb * 8192, &tm_v, cb * 64, hh, ts, bar_tma);
     }
-    if (CHANNEL) tma_load_3d(sG, &tm_g, 0, h, t0, bar_tma);
+    if (CHANNEL) tma_load_3d(sG, &tm_g, 0, hh, ts, bar_tma);
+  };
+  auto prefetch_l2 = [&](int w) {  // thread 0: a later item's tiles into L2
+    const int ck = w / H_v, hh = w - ck * H_v, hkk = hh / (H_v / H_qk);
+    const int ts = tab[ck].start;
+#pragma unroll
+    for (int cb = 0; cb < 2; ++cb) {
+      tma_prefetch_l2_3d(&tm_q, cb * 64, hkk, ts);
+      tma_prefetch_l2_3d(&tm_k, cb * 64, hkk, ts);
+      tma_prefetch_l2_3d(&tm_v, cb * 64, hh, ts);
+    }
+    if (CHANNEL) tma_prefetch_l2_3d(&tm_g, 0, hh, ts);
+  };
+  if (tid == 0) {
+    issue_loads(work);
+    if (work + (int)gridDim.x < total) prefetch_l2(work + gridDim.x);
   }
+
+  for (int it = 0; work < total; ++it, work += gridDim.x) {
+  const int chunk = work / H_v, h = work - chunk * H_v;
+  const ChunkEntry ce = tab[chunk];
+  const int L = ce.len, t0 = ce.start;
+  unsigned char *slot = slots + ((size_t)chunk * H_v + h) * SLOT_BYTES;
+  const int next = work + gridDim.x;
+
   if (tid < C) {
     sBeta[tid] = (tid < L) ? __ldg(beta + (size_t)(t0 + tid) * H_v + h) : 0.f;
     if (!CHANNEL) sGsc[tid] = (tid < L) ? __ldg(g_scalar + (size_t)(t0 + tid) * H_v + h) : 0.f;
   }
-  mbar_wait(bar_tma, 0, hdr, KDA_DEVICE_TIMEOUT);
+  mbar_wait(bar_tma, it & 1, hdr, KDA_DEVICE_TIMEOUT);
   __syncthreads();
 
   // ---- 2. per-token decays a = e^{g} (rows >= L: no decay), sub-chunk sums ----
-  // Thread (I, p) owns channels c = 2p, 2p+1 of the 16 tokens of sub-chunk I.
-  // Every in-chunk factor is a product of these a's: with G the in-chunk
-  // cumulative log-decay and E_I its value at the end of sub-chunk I,
+  // Thread (I, p, h) owns channels c = 2p, 2p+1 of tokens 8h .. 8h+7 of
+  // sub-chunk I; its neighbour lane (h ^ 1) owns the other half.  Every
+  // in-chunk factor is a product of these a's: with G the in-chunk cumulative
+  // log-decay and E_I its value at the end of sub-chunk I,
   //   e^{G_t - E_{I-1}} = prefix product of a in sub-chunk I up to t   (<= 1)
   //   e^{E_I - G_t}     = suffix product after t                       (<= 1)
   // and factors across sub-chunks are products of whole-sub-chunk products.
-  const int bI = tid >> 6, c2 = (tid & 63) * 2;
-  float a0[16], a1[16];
+  const int bI = tid >> 7, c2 = ((tid >> 1) & 63) * 2, rh = tid & 1;
+  float a0[8], a1[8];
+  float pre0, pre1, suf0, suf1;  // product of a before / after this thread's rows
   {
     float s0 = 0.f, s1 = 0.f, p0 = 1.f, p1 = 1.f;
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      const int t = 16 * bI + r;
+    for (int r = 0; r < 8; ++r) {
+      const int t = 16 * bI + 8 * rh + r;
       float g0 = 0.f, g1 = 0.f;
       if (t < L) {
         if (CHANNEL) {
@@ -320,10 +348,18 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       p0 *= a0[r];
       p1 *= a1[r];
     }
-    sPblk[bI * DK + c2] = p0;
-    sPblk[bI * DK + c2 + 1] = p1;
-    sGsum[bI * DK + c2] = s0;
-    sGsum[bI * DK + c2 + 1] = s1;
+    const float op0 = __shfl_xor_sync(0xffffffffu, p0, 1), op1 = __shfl_xor_sync(0xffffffffu, p1, 1);
+    const float os0 = __shfl_xor_sync(0xffffffffu, s0, 1), os1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+    pre0 = rh ? op0 : 1.f;
+    pre1 = rh ? op1 : 1.f;
+    suf0 = rh ? 1.f : op0;
+    suf1 = rh ? 1.f : op1;
+    if (rh == 0) {
+      sPblk[bI * DK + c2] = p0 * op0;
+      sPblk[bI * DK + c2 + 1] = p1 * op1;
+      sGsum[bI * DK + c2] = s0 + os0;
+      sGsum[bI * DK + c2 + 1] = s1 + os1;
+    }
   }
   __syncthreads();  // g is consumed: its region is reused below
 
@@ -359,23 +395,23 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       F0[J] = f0;
       F1[J] = f1;
     }
-    if (bI == 0) {
+    if (bI == 0 && rh == 0) {
       sGLe[c2] = ge0 * sPblk[c2];  // e^{G_L}: product over all four sub-chunks
       sGLe[c2 + 1] = ge1 * sPblk[c2 + 1];
     }
     // suffix products e^{E_I - G_t}
-    float w0[16], w1[16];
-    w0[15] = 1.f;
-    w1[15] = 1.f;
+    float w0[8], w1[8];
+    w0[7] = suf0;
+    w1[7] = suf1;
 #pragma unroll
-    for (int r = 14; r >= 0; --r) {
+    for (int r = 6; r >= 0; --r) {
       w0[r] = w0[r + 1] * a0[r + 1];
       w1[r] = w1[r + 1] * a1[r + 1];
     }
-    float pq0 = 1.f, pq1 = 1.f;  // prefix product through t-1: e^{Gp_t - E_{I-1}}
+    float pq0 = pre0, pq1 = pre1;  // prefix product through t-1: e^{Gp_t - E_{I-1}}
 #pragma unroll
-    for (int r = 0; r < 16; ++r) {
-      const int t = 16 * bI + r;
+    for (int r = 0; r < 8; ++r) {
+      const int t = 16 * bI + 8 * rh + r;
       const uint32_t koff = (c2 >> 6) * 8192 + kmajor_off(t, c2 & 63);
       const uint32_t kraw = *reinterpret_cast<const uint32_t *>(sK + koff);
       const uint32_t qraw = *reinterpret_cast<const uint32_t *>(sQ + koff);
@@ -389,7 +425,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float re0 = rw0 * a0[r], re1 = rw1 * a1[r];       // e^{E_I - Gp_t}
       pq0 = bq0;
       pq1 = bq1;
-      const int rowK = 32 * bI + r, rowQ = rowK + 16;
+      const int rowK = 32 * bI + 8 * rh + r, rowQ = rowK + 16;
       // Gram right operand (keys scaled to their sub-chunk end)
       const uint32_t rb = X_R + (c2 >> 6) * 16384;
       *reinterpret_cast<uint32_t *>(sX + rb + kmajor_off(rowK, c2 & 63)) = pack_bf16x2(k0 * rw0, k1 * rw1);
@@ -437,8 +473,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   mbar_wait(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
 
-  const int quad = warp & 3, half = warp >> 2;
-  const int lane_row = 32 * quad + lane;  // TMEM lane this thread reads
+  // readbacks: warp (quad, qtr) reads TMEM lanes 32*quad .. +31, column quarter qtr
+  const int quad = warp & 3, qtr = warp >> 2;
+  const int lane_row = 32 * quad + lane;
 
   // ---- 5. Gram readback: masked, beta-scaled, into the next operands ----
   {
@@ -446,9 +483,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const bool isK = s < 16;
     const int i = 16 * I + (s & 15);
     float* nae = reinterpret_cast<float *>(sX + X_NAE);
-#pragma unroll
-    for (int part = 0; part < 2; ++part) {
-      const int J = 2 * half + part;
+    {
+      const int J = qtr;
       float v[32];
       tmem_ld32(taddr(tm, 32 * quad, TM_GRAM + 32 * J), v);
       tmem_ld_wait();
@@ -522,56 +558,43 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     __syncthreads();
     // (b) 32x32 level: T^{-1}[2p+1][2p] = -T^{-1}[2p+1][2p+1] N[2p+1][2p] T^{-1}[2p][2p]
     {
-      const int pp = tid >> 7, r = (tid >> 3) & 15, cq = (tid & 7) * 2;
+      const int pp = tid >> 8, r = (tid >> 4) & 15, cc = tid & 15;
       const int R0 = 32 * pp + 16, C0 = 32 * pp;  // block row / column offsets
-      float acc0 = 0.f, acc1 = 0.f;
+      float acc = 0.f;
 #pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2) {
-        const float nv = nae[(R0 + r) * LDN + C0 + s2];
-        acc0 = fmaf(nv, tinv[(C0 + s2) * LDN + C0 + cq], acc0);
-        acc1 = fmaf(nv, tinv[(C0 + s2) * LDN + C0 + cq + 1], acc1);
-      }
-      tmp[(16 * pp + r) * 32 + cq] = acc0;
-      tmp[(16 * pp + r) * 32 + cq + 1] = acc1;
+      for (int s2 = 0; s2 < 16; ++s2)
+        acc = fmaf(nae[(R0 + r) * LDN + C0 + s2], tinv[(C0 + s2) * LDN + C0 + cc], acc);
+      tmp[(16 * pp + r) * 32 + cc] = acc;
       __syncthreads();
-      acc0 = acc1 = 0.f;
+      acc = 0.f;
 #pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2) {
-        const float tv = tinv[(R0 + r) * LDN + R0 + s2];
-        acc0 = fmaf(tv, tmp[(16 * pp + s2) * 32 + cq], acc0);
-        acc1 = fmaf(tv, tmp[(16 * pp + s2) * 32 + cq + 1], acc1);
-      }
-      tinv[(R0 + r) * LDN + C0 + cq] = -acc0;
-      tinv[(R0 + r) * LDN + C0 + cq + 1] = -acc1;
+      for (int s2 = 0; s2 < 16; ++s2)
+        acc = fmaf(tinv[(R0 + r) * LDN + R0 + s2], tmp[(16 * pp + s2) * 32 + cc], acc);
+      tinv[(R0 + r) * LDN + C0 + cc] = -acc;
       __syncthreads();
     }
     // (c) 64x64 level: T^{-1}[lo][hi] = -T^{-1}[lo][lo] N[lo][hi] T^{-1}[hi][hi] (32x32 blocks)
     {
-      const int r = tid >> 3, cq = (tid & 7) * 4;
-      float acc[4] = {0.f, 0.f, 0.f, 0.f};
+      const int r = tid >> 4, cq = (tid & 15) * 2;
+      float acc0 = 0.f, acc1 = 0.f;
 #pragma unroll 8
       for (int s2 = 0; s2 < 32; ++s2) {
         const float nv = nae[(32 + r) * LDN + s2];
-        const float4 tv = *reinterpret_cast<const float4 *>(tinv + s2 * LDN + cq);
-        acc[0] = fmaf(nv, tv.x, acc[0]);
-        acc[1] = fmaf(nv, tv.y, acc[1]);
-        acc[2] = fmaf(nv, tv.z, acc[2]);
-        acc[3] = fmaf(nv, tv.w, acc[3]);
+        const float2 tv = *reinterpret_cast<const float2 *>(tinv + s2 * LDN + cq);
+        acc0 = fmaf(nv, tv.x, acc0);
+        acc1 = fmaf(nv, tv.y, acc1);
       }
-      *reinterpret_cast<float4 *>(tmp + r * 32 + cq) = make_float4(acc[0], acc[1], acc[2], acc[3]);
+      *reinterpret_cast<float2 *>(tmp + r * 32 + cq) = make_float2(acc0, acc1);
       __syncthreads();
-      acc[0] = acc[1] = acc[2] = acc[3] = 0.f;
+      acc0 = acc1 = 0.f;
 #pragma unroll 8
       for (int s2 = 0; s2 < 32; ++s2) {
         const float tv = tinv[(32 + r) * LDN + 32 + s2];
-        const float4 xv = *reinterpret_cast<const float4 *>(tmp + s2 * 32 + cq);
-        acc[0] = fmaf(tv, xv.x, acc[0]);
-        acc[1] = fmaf(tv, xv.y, acc[1]);
-        acc[2] = fmaf(tv, xv.z, acc[2]);
-        acc[3] = fmaf(tv, xv.w, acc[3]);
+        const float2 xv = *reinterpret_cast<const float2 *>(tmp + s2 * 32 + cq);
+        acc0 = fmaf(tv, xv.x, acc0);
+        acc1 = fmaf(tv, xv.y, acc1);
       }
-      *reinterpret_cast<float4 *>(tinv + (32 + r) * LDN + cq) =
-          make_float4(-acc[0], -acc[1], -acc[2], -acc[3]);
+      *reinterpret_cast<float2 *>(tinv + (32 + r) * LDN + cq) = make_float2(-acc0, -acc1);
       __syncthreads();
     }
     // bf16 copy, K-major [i][j]
@@ -608,24 +631,20 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   // readback W (lanes c, cols i) -> K-major [c][t]; Y (lanes n, cols i) -> K-major [n][t]
   {
-    float v[32];
-    tmem_ld32(taddr(tm, 32 * quad, TM_W + 32 * half), v);
+    float v[16], v2[16];
+    tmem_ld16(taddr(tm, 32 * quad, TM_W + 16 * qtr), v);
+    tmem_ld16(taddr(tm, 32 * quad, TM_YB + 16 * qtr), v2);
     tmem_ld_wait();
 #pragma unroll
-    for (int seg = 0; seg < 4; ++seg) {
-      float x[8];
+    for (int seg = 0; seg < 2; ++seg) {
+      float x[8], y[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = v[8 * seg + u];
-      st16(sX + X_W + kmajor_off(lane_row, 32 * half + 8 * seg), pack8(x));
-    }
-    tmem_ld32(taddr(tm, 32 * quad, TM_YB + 32 * half), v);
-    tmem_ld_wait();
-#pragma unroll
-    for (int seg = 0; seg < 4; ++seg) {
-      float x[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = v[8 * seg + u];
-      st16(sX + X_Y + kmajor_off(lane_row, 32 * half + 8 * seg), pack8(x));
+      for (int u = 0; u < 8; ++u) {
+        x[u] = v[8 * seg + u];
+        y[u] = v2[8 * seg + u];
+      }
+      st16(sX + X_W + kmajor_off(lane_row, 16 * qtr + 8 * seg), pack8(x));
+      st16(sX + X_Y + kmajor_off(lane_row, 16 * qtr + 8 * seg), pack8(y));
     }
   }
   fence_async_smem();
@@ -657,49 +676,44 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   {
     float v[32];
     // U (lanes n, cols t) -> K-major [n][t]
-    tmem_ld32(taddr(tm, 32 * quad, TM_U + 32 * half), v);
+    float u16[16], x16[16];
+    tmem_ld16(taddr(tm, 32 * quad, TM_U + 16 * qtr), u16);
+    tmem_ld32(taddr(tm, 32 * quad, TM_P + 32 * qtr), v);
+    tmem_ld16(taddr(tm, 32 * quad, TM_X + 16 * qtr), x16);
     tmem_ld_wait();
 #pragma unroll
-    for (int seg = 0; seg < 4; ++seg) {
+    for (int seg = 0; seg < 2; ++seg) {
       float x[8];
 #pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = v[8 * seg + u];
-      st16(sX + X_U + kmajor_off(lane_row, 32 * half + 8 * seg), pack8(x));
+      for (int u = 0; u < 8; ++u) x[u] = u16[8 * seg + u];
+      st16(sX + X_U + kmajor_off(lane_row, 16 * qtr + 8 * seg), pack8(x));
     }
     // P = Diag(e^{G_L}) - K_b^T beta W (lanes i, cols c) -> K-major A image [i][c]
     const int i = lane_row;
     const float gl = sGLe[i];
 #pragma unroll
-    for (int part = 0; part < 2; ++part) {
-      const int c0 = 64 * half + 32 * part;
-      tmem_ld32(taddr(tm, 32 * quad, TM_P + c0), v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int seg = 0; seg < 4; ++seg) {
-        float x[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const int c = c0 + 8 * seg + u;
-          x[u] = (c == i ? gl : 0.f) - v[8 * seg + u];
-        }
-        const int c = c0 + 8 * seg;
-        st16(sX + X_PI + (c >> 6) * 16384 + kmajor_off(i, c & 63), pack8(x));
-      }
-    }
-    // Q'[t][c] = q_tc e^{G_tc} - X[c][t] (lanes c, cols t) -> MN-major A image [c][t]
-    const int c = lane_row;
-    tmem_ld32(taddr(tm, 32 * quad, TM_X + 32 * half), v);
-    tmem_ld_wait();
-#pragma unroll
     for (int seg = 0; seg < 4; ++seg) {
       float x[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        const int t = 32 * half + 8 * seg + u;
-        const float qg = ld_bf16(sQ, (c >> 6) * 8192 + kmajor_off(t, c & 63));  // q e^{G}
-        x[u] = (t < L) ? qg - v[8 * seg + u] : 0.f;
+        const int c = 32 * qtr + 8 * seg + u;
+        x[u] = (c == i ? gl : 0.f) - v[8 * seg + u];
       }
-      st16(sX + X_QPI + sw128((uint32_t)(c * 128 + (32 * half + 8 * seg) * 2)), pack8(x));
+      const int c = 32 * qtr + 8 * seg;
+      st16(sX + X_PI + (c >> 6) * 16384 + kmajor_off(i, c & 63), pack8(x));
+    }
+    // Q'[t][c] = q_tc e^{G_tc} - X[c][t] (lanes c, cols t) -> MN-major A image [c][t]
+    const int c = lane_row;
+#pragma unroll
+    for (int seg = 0; seg < 2; ++seg) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int t = 16 * qtr + 8 * seg + u;
+        const float qg = ld_bf16(sQ, (c >> 6) * 8192 + kmajor_off(t, c & 63));  // q e^{G}
+        x[u] = (t < L) ? qg - x16[8 * seg + u] : 0.f;
+      }
+      st16(sX + X_QPI + sw128((uint32_t)(c * 128 + (16 * qtr + 8 * seg) * 2)), pack8(x));
     }
   }
   fence_async_smem();
@@ -736,34 +750,35 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   mbar_wait(bar_mma, 1, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
 
+  // the input tiles are consumed: start the next item's loads now
+  if (tid == 0 && next < total) {
+    issue_loads(next);
+    if (next + (int)gridDim.x < total) prefetch_l2(next + gridDim.x);
+  }
   if (tid == 0) bulk_wait_read0();  // the P / Q' images may now be overwritten
   __syncthreads();
   {
     float v[32];
     // O_intra^T (lanes j, cols t) -> image row-major [j][t]
     const int j = lane_row;
-    tmem_ld32(taddr(tm, 32 * quad, TM_OI + 32 * half), v);
+    float o16[16];
+    tmem_ld16(taddr(tm, 32 * quad, TM_OI + 16 * qtr), o16);
+    tmem_ld32(taddr(tm, 32 * quad, TM_QC + 32 * qtr), v);
     tmem_ld_wait();
+#pragma unroll
+    for (int seg = 0; seg < 2; ++seg) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = o16[8 * seg + u];
+      st16(sX + X_OII + rowimg_off(j, C * 2, 2 * qtr + seg), pack8(x));
+    }
+    // Qc^T (lanes j, cols i) -> image row-major [j][i]
 #pragma unroll
     for (int seg = 0; seg < 4; ++seg) {
       float x[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) x[u] = v[8 * seg + u];
-      st16(sX + X_OII + rowimg_off(j, C * 2, 4 * half + seg), pack8(x));
-    }
-    // Qc^T (lanes j, cols i) -> image row-major [j][i]
-#pragma unroll
-    for (int part = 0; part < 2; ++part) {
-      const int i0 = 64 * half + 32 * part;
-      tmem_ld32(taddr(tm, 32 * quad, TM_QC + i0), v);
-      tmem_ld_wait();
-#pragma unroll
-      for (int seg = 0; seg < 4; ++seg) {
-        float x[8];
-#pragma unroll
-        for (int u = 0; u < 8; ++u) x[u] = v[8 * seg + u];
-        st16(sX + X_PI + rowimg_off(j, DK * 2, i0 / 8 + seg), pack8(x));
-      }
+      st16(sX + X_PI + rowimg_off(j, DK * 2, 4 * qtr + seg), pack8(x));
     }
   }
   fence_async_smem();
@@ -773,8 +788,16 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     bulk_s2g(slot + SLOT_QC, sX + X_PI, 32768);
     bulk_s2g(slot + SLOT_OI, sX + X_OII, 16384);
     bulk_commit();
-    bulk_wait0();
+    bulk_wait_read0();  // the next item rebuilds over these images
   }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  }  // work items
+
+  if (tid == 0) bulk_wait0();
+  tc_fence_before();
+  __syncthreads();
   if (warp == 0) tmem_dealloc(tm, 512);
 }
 
@@ -813,8 +836,9 @@ chunk_scan_kernel(const int32_t *hdr, const int32_t *__restrict__ seq_off,
                   __nv_bfloat16 *__restrict__ o, const float *__restrict__ s0,
                   float *__restrict__ sT, int H_v, int32_t *err) {
   extern __shared__ unsigned char smem_raw[];
-  unsigned char *sm = reinterpret_cast<unsigned char *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
+  // 1024-byte aligned base, derived by pointer arithmetic on the shared array so
+  // that the compiler keeps shared-memory addressing for every access
+  unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
   uint64_t *full = reinterpret_cast<uint64_t *>(sm + SC_MISC);  // [NSTAGE]
   uint64_t *empty = full + NSTAGE;                              // [NSTAGE], chain + out arrivals
   uint64_t *op_ready = empty + NSTAGE;                          // [3], chain arrivals
@@ -1008,6 +1032,13 @@ chunk_scan_kernel(const int32_t *hdr, const int32_t *__restrict__ seq_off,
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
+
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -1083,7 +1114,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
   auto prep = a.channel_gate ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
   e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM);
   if (e != cudaSuccess) return e;
-  dim3 gp((unsigned)max_chunks, (unsigned)a.H_v);
+  const int64_t items = max_chunks * a.H_v;
+  dim3 gp((unsigned)(items < sm_count() ? items : sm_count()));
   {
     TraceScope tr("chunk_prep_kernel", stream);
     prep<<<gp, kPrepThreads, PREP_SMEM, stream>>>(mq, mk, mv, mg, a.channel_gate ? nullptr : a.g,

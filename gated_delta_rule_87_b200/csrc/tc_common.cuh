@@ -46,22 +46,25 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
 
+// One poll: the thread may sleep (up to kSuspendNs) until the phase
+// completes, so a waiting warp does not spin on issue slots.
+constexpr uint32_t kSuspendNs = 1000000;
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(kSuspendNs)
       : "memory");
   return ok != 0;
 }
 
-// Upper bound on polls of one mbarrier phase.  try_wait suspends the thread
-// for a hardware-defined interval per poll, so this is far above any
-// legitimate wait (seconds) while still ending a wait that can never finish.
-constexpr uint32_t kMaxPolls = 1u << 24;
+// Upper bound on polls of one mbarrier phase (about kMaxPolls x 1 ms, i.e.
+// seconds): far above any legitimate wait, but a wait that can never finish
+// still ends.
+constexpr uint32_t kMaxPolls = 4096;
 
 // Wait for the phase with the given parity to complete.  Returns false (and
 // raises *err, when given) if the bound is hit; the caller then skips its
@@ -119,6 +122,13 @@ __device__ __forceinline__ void tma_load_3d(void *dst_smem, const CUtensorMap *m
       ::"r"(smem_u32(dst_smem)), "l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2),
       "r"(smem_u32(bar))
       : "memory");
+}
+
+// Prefetch one tile of a tensor map into L2 (no shared-memory destination).
+__device__ __forceinline__ void tma_prefetch_l2_3d(const CUtensorMap *map, int c0, int c1, int c2) {
+  asm volatile("cp.async.bulk.prefetch.tensor.3d.L2.global.tile [%0, {%1, %2, %3}];"
+               ::"l"(reinterpret_cast<uint64_t>(map)), "r"(c0), "r"(c1), "r"(c2)
+               : "memory");
 }
 
 __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap *map) {
