@@ -426,7 +426,7 @@ def bench_decode(args, device, world, peaks, stream, flush):
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
                          "traffic": None, "peak_source": peaks["source"],
-                         "kernel": "decode_step_kernel"},
+                         "kernel": "recurrent_kernel"},
             "l2": "state (512 MB) larger than L2; not flushed",
             "launches": w.steps}
 

@@ -21,8 +21,9 @@ from typing import Optional, Tuple
 
 __all__ = [
     "lib", "library_path", "KdaError", "kda_chunk_fwd", "gdn_chunk_fwd", "kda_decode_step",
-    "gdn_decode_step", "chunk_workspace_size", "check_device_status", "EXPORTED_SYMBOLS",
-    "trace_enable", "trace_read",
+    "gdn_decode_step", "kda_recurrent_fwd", "gdn_recurrent_fwd", "state_gather", "state_scatter",
+    "chunk_workspace_size", "check_device_status", "EXPORTED_SYMBOLS",
+    "trace_enable", "trace_read", "ERASE_THEN_DECAY", "DECAY_THEN_ERASE",
     "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
     "KDA_ERR_DEVICE_CHECK", "KDA_ERR_WORKSPACE",
 ]
@@ -33,19 +34,31 @@ library_path = os.path.join(_PKG, "libgated_delta.so")
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_DEVICE_CHECK, \
     KDA_ERR_WORKSPACE = range(6)
 KDA_F32, KDA_BF16 = 0, 1
+# decay order (KDA): the table's literal order, or the decay applied before the erase
+ERASE_THEN_DECAY, DECAY_THEN_ERASE = "erase_then_decay", "decay_then_erase"
+_ORDER = {ERASE_THEN_DECAY: 0, DECAY_THEN_ERASE: 1}
 
 EXPORTED_SYMBOLS = (
     "kda_chunk_fwd", "kda_chunk_fwd_workspace_size", "gdn_chunk_fwd",
     "gdn_chunk_fwd_workspace_size", "kda_decode_step", "gdn_decode_step",
     "kda_check_device_status", "kda_status_string", "kda_last_error", "kda_abi_version",
-    "kda_trace_enable", "kda_trace_read", "kda_chunk_fwd_noalloc",
+    "kda_trace_enable", "kda_trace_read", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_ex",
+    "gdn_chunk_fwd_ex", "kda_recurrent_fwd", "gdn_recurrent_fwd", "kda_state_gather",
+    "kda_state_scatter",
 )
 
 _lock = threading.Lock()
 _lib = None
 
 _vp, _fp, _i32, _sz = ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_size_t
+_i64, _int = ctypes.c_int64, ctypes.c_int
 _SIGS = {
+    "kda_chunk_fwd_ex": ([_vp] * 9 + [_i64, _vp] + [_i32] * 6 + [_int, _int, _vp, _sz, _vp], _int),
+    "gdn_chunk_fwd_ex": ([_vp] * 9 + [_i64, _vp] + [_i32] * 7 + [_int, _vp, _sz, _vp], _int),
+    "kda_recurrent_fwd": ([_vp] * 8 + [_i64] + [_i32] * 5 + [_int, _int, _vp], _int),
+    "gdn_recurrent_fwd": ([_vp] * 8 + [_i64] + [_i32] * 6 + [_int, _vp], _int),
+    "kda_state_gather": ([_vp, _vp, _i64, _vp] + [_i32] * 4 + [_vp], _int),
+    "kda_state_scatter": ([_vp, _vp, _vp, _i64] + [_i32] * 4 + [_vp], _int),
     "kda_chunk_fwd": ([_vp] * 9 + [_i32] * 6 + [ctypes.c_int, _vp, _sz, _vp], ctypes.c_int),
     "gdn_chunk_fwd": ([_vp] * 9 + [_i32] * 7 + [ctypes.c_int, _vp, _sz, _vp], ctypes.c_int),
     "kda_chunk_fwd_workspace_size": ([_i32] * 6 + [ctypes.c_int], _sz),
@@ -147,8 +160,28 @@ def _alloc_workspace(nbytes: int, device):
     return torch.empty(max(nbytes, 256), dtype=torch.uint8, device=device)
 
 
+def _order_code(order) -> int:
+    if order not in _ORDER:
+        raise ValueError(f"order must be one of {sorted(_ORDER)}, got {order!r}")
+    return _ORDER[order]
+
+
+def _slots(state_slots, state_pool, N):
+    torch = _torch()
+    if state_slots is None:
+        if state_pool is not None:
+            raise ValueError("state_pool needs state_slots")
+        return None, 0
+    if state_pool is None:
+        raise ValueError("state_slots needs state_pool")
+    if state_slots.dtype != torch.int32 or state_slots.numel() != N:
+        raise ValueError(f"state_slots must be int32 with {N} entries")
+    return state_slots, state_pool.shape[0]
+
+
 def _chunk_fwd(gate, q, k, v, g, beta, initial_state, cu_seqlens, output_final_state,
-               o, final_state, workspace, stream):
+               o, final_state, workspace, stream, order=ERASE_THEN_DECAY, state_pool=None,
+               state_slots=None):
     torch = _torch()
     if q.dim() != 4:
         raise ValueError("q, k, v must be [B, T, H, d]")
@@ -167,7 +200,14 @@ def _chunk_fwd(gate, q, k, v, g, beta, initial_state, cu_seqlens, output_final_s
     dev = q.device
     if o is None:
         o = torch.empty((B, T, H_v, d_v), dtype=q.dtype, device=dev)
-    if final_state is None and output_final_state:
+    slots, num_slots = _slots(state_slots, state_pool, N)
+    if slots is not None:
+        # pool mode: read and update pool[state_slots[n]] in place
+        if initial_state is not None or final_state is not None:
+            raise ValueError("with state_pool, pass neither initial_state nor final_state")
+        _f32(state_pool, "state_pool")
+        initial_state = final_state = state_pool
+    elif final_state is None and output_final_state:
         final_state = torch.empty((N, H_v, d_k, d_v), dtype=torch.float32, device=dev)
     need = chunk_workspace_size(B, T, H_qk, H_v, d_k, d_v, N if cu_seqlens is not None else 0,
                                 io, gate)
@@ -175,38 +215,45 @@ def _chunk_fwd(gate, q, k, v, g, beta, initial_state, cu_seqlens, output_final_s
         workspace = _alloc_workspace(need, dev)
     L = lib()
     args_common = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(o), _ptr(initial_state),
-                   _ptr(final_state), _ptr(cu_seqlens), N]
+                   _ptr(final_state), _ptr(slots), num_slots, _ptr(cu_seqlens), N]
     sh = _stream_handle(stream, dev)
     if gate == "channel":
-        st = L.kda_chunk_fwd(*args_common, B, T, H_v, d_k, d_v, io, _ptr(workspace),
-                             workspace.numel(), sh)
-        _check(st, "kda_chunk_fwd")
+        st = L.kda_chunk_fwd_ex(*args_common, B, T, H_v, d_k, d_v, _order_code(order), io,
+                                _ptr(workspace), workspace.numel(), sh)
+        _check(st, "kda_chunk_fwd_ex")
     else:
-        st = L.gdn_chunk_fwd(*args_common, B, T, H_qk, H_v, d_k, d_v, io, _ptr(workspace),
-                             workspace.numel(), sh)
-        _check(st, "gdn_chunk_fwd")
+        st = L.gdn_chunk_fwd_ex(*args_common, B, T, H_qk, H_v, d_k, d_v, io, _ptr(workspace),
+                                workspace.numel(), sh)
+        _check(st, "gdn_chunk_fwd_ex")
     return o, final_state, workspace
 
 
 def kda_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *,
                   output_final_state: bool = True, o=None, final_state=None, workspace=None,
-                  stream=None):
+                  stream=None, order: str = ERASE_THEN_DECAY, state_pool=None,
+                  state_slots=None):
     """KDA prefill.  q, k [B,T,H,d_k]; v [B,T,H,d_v] (bf16 or fp32); g [B,T,H,d_k]
     fp32 log-decay; beta [B,T,H] fp32; initial_state [N,H,d_k,d_v] fp32 or None;
     cu_seqlens int32 [N+1] (device) for packed sequences with B = 1.
-    Returns (o, final_state, workspace)."""
+    ``order`` places the decay after (default) or before the erase.  With
+    ``state_pool`` [num_slots,H,d_k,d_v] and ``state_slots`` int32 [N], sequence
+    n starts from pool[state_slots[n]] and its final state is written back
+    there (slots outside the pool: start from zeros, no final state).
+    Returns (o, final_state, workspace); final_state is the pool in pool mode."""
     return _chunk_fwd("channel", q, k, v, g, beta, initial_state, cu_seqlens,
-                      output_final_state, o, final_state, workspace, stream)
+                      output_final_state, o, final_state, workspace, stream, order, state_pool,
+                      state_slots)
 
 
 def gdn_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *,
                   output_final_state: bool = True, o=None, final_state=None, workspace=None,
-                  stream=None):
+                  stream=None, state_pool=None, state_slots=None):
     """Gated DeltaNet prefill.  q, k [B,T,H_qk,d_k]; v [B,T,H_v,d_v]; g, beta
-    [B,T,H_v] fp32 (scalar log-decay per head-token).  Returns (o, final_state,
-    workspace)."""
+    [B,T,H_v] fp32 (scalar log-decay per head-token).  ``state_pool`` /
+    ``state_slots`` as in kda_chunk_fwd.  Returns (o, final_state, workspace)."""
     return _chunk_fwd("scalar", q, k, v, g, beta, initial_state, cu_seqlens,
-                      output_final_state, o, final_state, workspace, stream)
+                      output_final_state, o, final_state, workspace, stream, ERASE_THEN_DECAY,
+                      state_pool, state_slots)
 
 
 def _decode(gate, q, k, v, g, beta, state, o, stream):
@@ -225,6 +272,73 @@ def _decode(gate, q, k, v, g, beta, state, o, stream):
     else:
         _check(L.gdn_decode_step(*ptrs, N, H_qk, H_v, d_k, d_v, io, sh), "gdn_decode_step")
     return o
+
+
+def _recurrent(gate, q, k, v, g, beta, state, state_slots, order, o, stream):
+    torch = _torch()
+    if q.dim() != 4:
+        raise ValueError("q, k, v must be [N, T, H, d]")
+    N, T, H_qk, d_k = q.shape
+    H_v, d_v = v.shape[2], v.shape[3]
+    io = _dtype_code(q)
+    _f32(g, "g"), _f32(beta, "beta"), _f32(state, "state")
+    slots, num_slots = _slots(state_slots, state if state_slots is not None else None, N)
+    if o is None:
+        o = torch.empty((N, T, H_v, d_v), dtype=q.dtype, device=q.device)
+    L = lib()
+    sh = _stream_handle(stream, q.device)
+    ptrs = [_ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta), _ptr(o), _ptr(state), _ptr(slots)]
+    if gate == "channel":
+        _check(L.kda_recurrent_fwd(*ptrs, num_slots, N, T, H_v, d_k, d_v, _order_code(order), io,
+                                   sh), "kda_recurrent_fwd")
+    else:
+        _check(L.gdn_recurrent_fwd(*ptrs, num_slots, N, T, H_qk, H_v, d_k, d_v, io, sh),
+               "gdn_recurrent_fwd")
+    return o
+
+
+def kda_recurrent_fwd(q, k, v, g, beta, state, *, state_slots=None,
+                      order: str = ERASE_THEN_DECAY, o=None, stream=None):
+    """T tokens for each of N sequences, token by token, state updated in place
+    (read once, written once).  q, k [N,T,H,d_k]; v [N,T,H,d_v]; g [N,T,H,d_k];
+    beta [N,T,H].  ``state`` is [N,H,d_k,d_v], or a pool [num_slots,H,d_k,d_v]
+    indexed by ``state_slots`` (int32 [N]; a slot outside the pool is a padding
+    entry: zero output, no state).  Returns o [N,T,H,d_v]."""
+    return _recurrent("channel", q, k, v, g, beta, state, state_slots, order, o, stream)
+
+
+def gdn_recurrent_fwd(q, k, v, g, beta, state, *, state_slots=None, o=None, stream=None):
+    """Gated DeltaNet form of kda_recurrent_fwd: q, k [N,T,H_qk,d_k]; v [N,T,H_v,d_v];
+    g, beta [N,T,H_v].  Returns o [N,T,H_v,d_v]."""
+    return _recurrent("scalar", q, k, v, g, beta, state, state_slots, ERASE_THEN_DECAY, o,
+                      stream)
+
+
+def state_gather(pool, state_slots, *, out=None, stream=None):
+    """out[n] = pool[state_slots[n]] (zeros for a slot outside the pool)."""
+    torch = _torch()
+    _f32(pool, "pool")
+    N = state_slots.numel()
+    _slots(state_slots, pool, N)
+    _, H, d_k, d_v = pool.shape
+    if out is None:
+        out = torch.empty((N, H, d_k, d_v), dtype=torch.float32, device=pool.device)
+    _check(lib().kda_state_gather(_ptr(pool), _ptr(state_slots), pool.shape[0], _ptr(out), N, H,
+                                  d_k, d_v, _stream_handle(stream, pool.device)),
+           "kda_state_gather")
+    return out
+
+
+def state_scatter(src, pool, state_slots, *, stream=None):
+    """pool[state_slots[n]] = src[n] (skipped for a slot outside the pool)."""
+    _f32(src, "src"), _f32(pool, "pool")
+    N = state_slots.numel()
+    _slots(state_slots, pool, N)
+    _, H, d_k, d_v = pool.shape
+    _check(lib().kda_state_scatter(_ptr(src), _ptr(pool), _ptr(state_slots), pool.shape[0], N, H,
+                                   d_k, d_v, _stream_handle(stream, pool.device)),
+           "kda_state_scatter")
+    return pool
 
 
 def kda_decode_step(q, k, v, g, beta, state, *, o=None, stream=None):

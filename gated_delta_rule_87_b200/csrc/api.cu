@@ -51,8 +51,11 @@ kda_status_t check_prefill(const gdr::PrefillArgs &a) {
   const void *ptrs16[] = {a.q, a.k, a.v, a.g, a.o, a.initial_state, a.final_state};
   for (const void *p : ptrs16)
     if (p && !aligned16(p)) return fail(KDA_ERR_INVALID_ARG, "pointer %p is not 16-byte aligned", p);
-  if ((a.beta && !aligned4(a.beta)) || (a.cu_seqlens && !aligned4(a.cu_seqlens)))
-    return fail(KDA_ERR_INVALID_ARG, "beta and cu_seqlens must be 4-byte aligned");
+  if ((a.beta && !aligned4(a.beta)) || (a.cu_seqlens && !aligned4(a.cu_seqlens)) ||
+      (a.state_slots && !aligned4(a.state_slots)))
+    return fail(KDA_ERR_INVALID_ARG, "beta, cu_seqlens and state_slots must be 4-byte aligned");
+  if (a.state_slots && a.num_slots < 0)
+    return fail(KDA_ERR_INVALID_ARG, "num_slots must be >= 0");
   if (a.cu_seqlens) {
     if (a.B != 1) return fail(KDA_ERR_INVALID_ARG, "packed sequences (cu_seqlens) need B == 1");
     if (a.num_seqs < 0) return fail(KDA_ERR_INVALID_ARG, "num_seqs must be >= 0");
@@ -81,6 +84,7 @@ kda_status_t run_prefill(gdr::PrefillArgs &a, cudaStream_t s) {
   cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, s);
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   if (!a.cu_seqlens) a.num_seqs = a.B;
+  if (!a.state_slots) a.num_slots = a.num_seqs;
   const bool tc = use_tensor_core_path(a);
   if (a.cu_seqlens && !tc) {  // the tensor-core path validates in its planning kernel
     e = gdr::launch_check_cu_seqlens(a.cu_seqlens, a.num_seqs, a.T, status, s);
@@ -88,7 +92,14 @@ kda_status_t run_prefill(gdr::PrefillArgs &a, cudaStream_t s) {
   }
   if (a.num_seqs == 0 || a.T == 0) {
     // nothing to compute; final state = initial state
-    if (a.final_state) {
+    const int64_t per_seq = (int64_t)a.H_v * a.d_k * a.d_v;
+    if (a.final_state && a.state_slots) {
+      if (a.final_state != a.initial_state) {
+        e = gdr::launch_state_copy(a.initial_state, a.state_slots, a.num_slots, a.final_state,
+                                   a.state_slots, a.num_slots, a.num_seqs, per_seq, s);
+        if (e != cudaSuccess) return cuda_fail(e, "final state copy");
+      }
+    } else if (a.final_state) {
       const size_t bytes = (size_t)a.num_seqs * a.H_v * a.d_k * a.d_v * sizeof(float);
       if (bytes) {
         e = a.initial_state ? cudaMemcpyAsync(a.final_state, a.initial_state, bytes,
@@ -110,6 +121,13 @@ kda_status_t run_prefill(gdr::PrefillArgs &a, cudaStream_t s) {
 namespace gdr {
 
 void set_last_error(const char *msg) { g_last_error = msg; }
+
+int sm_count() {
+  int dev = 0, n = 148;
+  if (cudaGetDevice(&dev) == cudaSuccess)
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+  return n > 0 ? n : 148;
+}
 
 __global__ void check_cu_seqlens_kernel(const int32_t *__restrict__ cu, int num_seqs, int T,
                                         int32_t *status) {
@@ -162,20 +180,56 @@ size_t gdn_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H_qk, int32_t 
   return gdr::prefill_workspace_bytes(B * T, H_v, d_k, d_v, n, io_dtype == KDA_BF16);
 }
 
+kda_status_t kda_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, void *o, const float *initial_state,
+                              float *final_state, const int32_t *state_slots, int64_t num_slots,
+                              const int32_t *cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                              int32_t H, int32_t d_k, int32_t d_v, kda_order_t order,
+                              kda_dtype_t io_dtype, void *workspace, size_t workspace_bytes,
+                              void *stream) {
+  if (io_dtype != KDA_F32 && io_dtype != KDA_BF16)
+    return fail(KDA_ERR_INVALID_ARG, "io_dtype must be KDA_F32 or KDA_BF16");
+  if (order != KDA_ERASE_THEN_DECAY && order != KDA_DECAY_THEN_ERASE)
+    return fail(KDA_ERR_INVALID_ARG, "order must be KDA_ERASE_THEN_DECAY or KDA_DECAY_THEN_ERASE");
+  gdr::PrefillArgs a{};
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = o;
+  a.initial_state = initial_state; a.final_state = final_state;
+  a.state_slots = state_slots; a.num_slots = num_slots;
+  a.cu_seqlens = cu_seqlens; a.num_seqs = cu_seqlens ? num_seqs : B;
+  a.B = B; a.T = T; a.H_qk = H; a.H_v = H; a.d_k = d_k; a.d_v = d_v;
+  a.channel_gate = true; a.decay_first = (order == KDA_DECAY_THEN_ERASE);
+  a.bf16 = (io_dtype == KDA_BF16);
+  a.workspace = workspace; a.workspace_bytes = workspace_bytes;
+  return run_prefill(a, static_cast<cudaStream_t>(stream));
+}
+
 kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
                            const float *beta, void *o, const float *initial_state,
                            float *final_state, const int32_t *cu_seqlens, int32_t num_seqs,
                            int32_t B, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
                            kda_dtype_t io_dtype, void *workspace, size_t workspace_bytes,
                            void *stream) {
+  return kda_chunk_fwd_ex(q, k, v, g, beta, o, initial_state, final_state, nullptr, 0,
+                          cu_seqlens, num_seqs, B, T, H, d_k, d_v, KDA_ERASE_THEN_DECAY, io_dtype,
+                          workspace, workspace_bytes, stream);
+}
+
+kda_status_t gdn_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *g,
+                              const float *beta, void *o, const float *initial_state,
+                              float *final_state, const int32_t *state_slots, int64_t num_slots,
+                              const int32_t *cu_seqlens, int32_t num_seqs, int32_t B, int32_t T,
+                              int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+                              kda_dtype_t io_dtype, void *workspace, size_t workspace_bytes,
+                              void *stream) {
   if (io_dtype != KDA_F32 && io_dtype != KDA_BF16)
     return fail(KDA_ERR_INVALID_ARG, "io_dtype must be KDA_F32 or KDA_BF16");
   gdr::PrefillArgs a{};
   a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = o;
   a.initial_state = initial_state; a.final_state = final_state;
+  a.state_slots = state_slots; a.num_slots = num_slots;
   a.cu_seqlens = cu_seqlens; a.num_seqs = cu_seqlens ? num_seqs : B;
-  a.B = B; a.T = T; a.H_qk = H; a.H_v = H; a.d_k = d_k; a.d_v = d_v;
-  a.channel_gate = true; a.bf16 = (io_dtype == KDA_BF16);
+  a.B = B; a.T = T; a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v;
+  a.channel_gate = false; a.bf16 = (io_dtype == KDA_BF16);
   a.workspace = workspace; a.workspace_bytes = workspace_bytes;
   return run_prefill(a, static_cast<cudaStream_t>(stream));
 }
@@ -186,27 +240,25 @@ kda_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const fl
                            int32_t B, int32_t T, int32_t H_qk, int32_t H_v, int32_t d_k,
                            int32_t d_v, kda_dtype_t io_dtype, void *workspace,
                            size_t workspace_bytes, void *stream) {
-  if (io_dtype != KDA_F32 && io_dtype != KDA_BF16)
-    return fail(KDA_ERR_INVALID_ARG, "io_dtype must be KDA_F32 or KDA_BF16");
-  gdr::PrefillArgs a{};
-  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = o;
-  a.initial_state = initial_state; a.final_state = final_state;
-  a.cu_seqlens = cu_seqlens; a.num_seqs = cu_seqlens ? num_seqs : B;
-  a.B = B; a.T = T; a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v;
-  a.channel_gate = false; a.bf16 = (io_dtype == KDA_BF16);
-  a.workspace = workspace; a.workspace_bytes = workspace_bytes;
-  return run_prefill(a, static_cast<cudaStream_t>(stream));
+  return gdn_chunk_fwd_ex(q, k, v, g, beta, o, initial_state, final_state, nullptr, 0,
+                          cu_seqlens, num_seqs, B, T, H_qk, H_v, d_k, d_v, io_dtype, workspace,
+                          workspace_bytes, stream);
 }
 
 static kda_status_t decode_common(gdr::DecodeArgs &a, kda_dtype_t io_dtype, void *stream) {
   if (io_dtype != KDA_F32 && io_dtype != KDA_BF16)
     return fail(KDA_ERR_INVALID_ARG, "io_dtype must be KDA_F32 or KDA_BF16");
   a.bf16 = (io_dtype == KDA_BF16);
-  if (a.N == 0 && a.H_qk > 0 && a.H_v > 0) return KDA_OK;  // empty batch: nothing to do
+  if (a.N < 0 || a.T < 0 || a.H_qk <= 0 || a.H_v <= 0)
+    return fail(KDA_ERR_INVALID_ARG, "need N >= 0, T >= 0 and H > 0");
+  if (a.N == 0 || a.T == 0) return KDA_OK;  // no tokens: nothing to do
   if (!a.q || !a.k || !a.v || !a.g || !a.beta || !a.o || !a.state)
     return fail(KDA_ERR_INVALID_ARG, "q, k, v, g, beta, o and state must be non-NULL");
-  if (a.N < 0 || a.H_qk <= 0 || a.H_v <= 0)
-    return fail(KDA_ERR_INVALID_ARG, "need N >= 0 and H > 0");
+  if (a.slots && (!aligned4(a.slots) || a.num_slots < 0))
+    return fail(KDA_ERR_INVALID_ARG, "state_slots must be 4-byte aligned and num_slots >= 0");
+  if (!a.slots) a.num_slots = a.N;
+  if ((int64_t)a.N * a.T > INT32_MAX)
+    return fail(KDA_ERR_INVALID_ARG, "N*T must fit in int32");
   if (a.H_v % a.H_qk != 0)
     return fail(KDA_ERR_INVALID_ARG, "H_v (%d) must be a multiple of H_qk (%d)", a.H_v, a.H_qk);
   if (!head_dim_ok(a.d_k) || !head_dim_ok(a.d_v))
@@ -224,28 +276,87 @@ static kda_status_t decode_common(gdr::DecodeArgs &a, kda_dtype_t io_dtype, void
     return fail(KDA_ERR_INVALID_ARG, "g and beta must be 4-byte aligned");
   if (a.o == a.q || a.o == a.k || a.o == a.v || a.o == a.state)
     return fail(KDA_ERR_INVALID_ARG, "o must not alias an input or the state");
-  cudaError_t e = gdr::launch_decode_step(a, static_cast<cudaStream_t>(stream));
-  if (e != cudaSuccess) return cuda_fail(e, "decode launch");
+  cudaError_t e = gdr::launch_recurrent(a, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "recurrent launch");
   return KDA_OK;
+}
+
+kda_status_t kda_recurrent_fwd(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, void *o, float *state,
+                               const int32_t *state_slots, int64_t num_slots, int32_t N,
+                               int32_t T, int32_t H, int32_t d_k, int32_t d_v, kda_order_t order,
+                               kda_dtype_t io_dtype, void *stream) {
+  if (order != KDA_ERASE_THEN_DECAY && order != KDA_DECAY_THEN_ERASE)
+    return fail(KDA_ERR_INVALID_ARG, "order must be KDA_ERASE_THEN_DECAY or KDA_DECAY_THEN_ERASE");
+  gdr::DecodeArgs a{};
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = o; a.state = state;
+  a.slots = state_slots; a.num_slots = num_slots;
+  a.N = N; a.T = T; a.H_qk = H; a.H_v = H; a.d_k = d_k; a.d_v = d_v; a.channel_gate = true;
+  a.decay_first = (order == KDA_DECAY_THEN_ERASE);
+  return decode_common(a, io_dtype, stream);
+}
+
+kda_status_t gdn_recurrent_fwd(const void *q, const void *k, const void *v, const float *g,
+                               const float *beta, void *o, float *state,
+                               const int32_t *state_slots, int64_t num_slots, int32_t N,
+                               int32_t T, int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
+                               kda_dtype_t io_dtype, void *stream) {
+  gdr::DecodeArgs a{};
+  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = o; a.state = state;
+  a.slots = state_slots; a.num_slots = num_slots;
+  a.N = N; a.T = T; a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v;
+  a.channel_gate = false;
+  return decode_common(a, io_dtype, stream);
 }
 
 kda_status_t kda_decode_step(const void *q, const void *k, const void *v, const float *g,
                              const float *beta, void *o, float *state, int32_t N, int32_t H,
                              int32_t d_k, int32_t d_v, kda_dtype_t io_dtype, void *stream) {
-  gdr::DecodeArgs a{};
-  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = o; a.state = state;
-  a.N = N; a.H_qk = H; a.H_v = H; a.d_k = d_k; a.d_v = d_v; a.channel_gate = true;
-  return decode_common(a, io_dtype, stream);
+  return kda_recurrent_fwd(q, k, v, g, beta, o, state, nullptr, 0, N, 1, H, d_k, d_v,
+                           KDA_ERASE_THEN_DECAY, io_dtype, stream);
 }
 
 kda_status_t gdn_decode_step(const void *q, const void *k, const void *v, const float *g,
                              const float *beta, void *o, float *state, int32_t N, int32_t H_qk,
                              int32_t H_v, int32_t d_k, int32_t d_v, kda_dtype_t io_dtype,
                              void *stream) {
-  gdr::DecodeArgs a{};
-  a.q = q; a.k = k; a.v = v; a.g = g; a.beta = beta; a.o = o; a.state = state;
-  a.N = N; a.H_qk = H_qk; a.H_v = H_v; a.d_k = d_k; a.d_v = d_v; a.channel_gate = false;
-  return decode_common(a, io_dtype, stream);
+  return gdn_recurrent_fwd(q, k, v, g, beta, o, state, nullptr, 0, N, 1, H_qk, H_v, d_k, d_v,
+                           io_dtype, stream);
+}
+
+static kda_status_t state_copy_common(const float *src, const int32_t *src_slots,
+                                      int64_t src_limit, float *dst, const int32_t *dst_slots,
+                                      int64_t dst_limit, int32_t N, int32_t H, int32_t d_k,
+                                      int32_t d_v, void *stream) {
+  if (N < 0 || H <= 0) return fail(KDA_ERR_INVALID_ARG, "need N >= 0 and H > 0");
+  if (!head_dim_ok(d_k) || !head_dim_ok(d_v))
+    return fail(KDA_ERR_UNSUPPORTED, "d_k and d_v must be 64 or 128 (got %d, %d)", d_k, d_v);
+  if (N == 0) return KDA_OK;
+  if (!src || !dst || !(src_slots || dst_slots))
+    return fail(KDA_ERR_INVALID_ARG, "pool, slots and the dense buffer must be non-NULL");
+  if (!aligned16(src) || !aligned16(dst))
+    return fail(KDA_ERR_INVALID_ARG, "state buffers must be 16-byte aligned");
+  if ((src_slots && !aligned4(src_slots)) || (dst_slots && !aligned4(dst_slots)))
+    return fail(KDA_ERR_INVALID_ARG, "slots must be 4-byte aligned");
+  if (src_limit < 0 || dst_limit < 0) return fail(KDA_ERR_INVALID_ARG, "num_slots must be >= 0");
+  if (src == dst) return fail(KDA_ERR_INVALID_ARG, "the pool and the dense buffer must differ");
+  const int64_t per_seq = (int64_t)H * d_k * d_v;
+  cudaError_t e = gdr::launch_state_copy(src, src_slots, src_limit, dst, dst_slots, dst_limit, N,
+                                         per_seq, static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "state copy launch");
+  return KDA_OK;
+}
+
+kda_status_t kda_state_gather(const float *pool, const int32_t *state_slots, int64_t num_slots,
+                              float *out, int32_t N, int32_t H, int32_t d_k, int32_t d_v,
+                              void *stream) {
+  return state_copy_common(pool, state_slots, num_slots, out, nullptr, N, N, H, d_k, d_v, stream);
+}
+
+kda_status_t kda_state_scatter(const float *src, float *pool, const int32_t *state_slots,
+                               int64_t num_slots, int32_t N, int32_t H, int32_t d_k, int32_t d_v,
+                               void *stream) {
+  return state_copy_common(src, nullptr, N, pool, state_slots, num_slots, N, H, d_k, d_v, stream);
 }
 
 kda_status_t kda_check_device_status(const void *workspace, void *stream, int32_t *device_code) {

@@ -1,23 +1,43 @@
-// One decode step of the gated delta rule, in place on the fp32 state.
+// Token-by-token (recurrent) form of the gated delta rule, in place on the
+// fp32 state: one decode step (T = 1) or a few tokens per sequence (T > 1:
+// speculative decoding, chunked prefill in small pieces).
 //
 // Operator: thethings.ai "The argument, in one page", table "Everything, in
 // one table", rows "KDA" / "Gated DeltaNet":
 //     S' = Diag(a) (S - beta k (k^T S)) + beta k v^T,   o = S'^T q.
 // Expanding the readout through the update lets one pass over the old state
-// produce everything:
+// produce everything a token needs:
 //     r = S^T k,   p = S^T (a . q)
 //     S' = a . (S - beta k r^T) + beta k v^T
 //     o  = p - beta (k . (a . q)) r + beta (k . q) v
-// so each state element is read once and written once.  The step is bound by
-// HBM bandwidth (about 1 flop per byte): the kernel is a streaming copy with
-// arithmetic in registers.
+// With the decay applied before the erase (the variant order, S' = (I - beta k
+// k^T) Diag(a) S + beta k v^T) the same pass reads r = S^T (a . k) instead:
+//     S' = a . S - beta k r^T + beta k v^T,   o = p - beta (k . q) r + beta (k . q) v.
+// Both orders are one template: per token and state row i the kernel keeps
+//     kr_i  the direction recall is read along   (k_i, or a_i k_i)
+//     e_i   the erase coefficient of row i        (beta a_i k_i, or beta k_i)
+// and c_r, the coefficient of r in the readout (beta k.(a.q), or beta k.q).
+//
+// The state is read from HBM once and written once per call, whatever T; the
+// T tokens are applied to it in registers.  A single step is bound by HBM
+// bandwidth (about 1 flop per byte): a streaming copy with arithmetic.
 //
 // Mapping: one CTA of 8 warps per (sequence, head).  Warp w owns rows
 // [w*D_K/8, (w+1)*D_K/8) of the d_k x d_v state; lane l owns columns
 // [l*D_V/32, (l+1)*D_V/32), loaded with one 16-byte (d_v = 128) or 8-byte
 // (d_v = 64) streaming load per row, so every warp load is a contiguous
 // 512-byte (256-byte) row.  The column sums r and p are reduced over the
-// rows of a warp in registers and across warps through shared memory.
+// rows of a warp in registers and across warps through shared memory.  Per
+// token there is one block barrier: the per-token vectors are triple-buffered
+// and the cross-warp partial sums double-buffered, so the next token's
+// vectors are written while the current token is still being applied.
+//
+// State pool: with a slot array the state of sequence n is pool[slots[n]]
+// (checkpointed recurrent states for serving, inferencex.semianalysis.com
+// "Linear attention", "Why it matters": a dropped state can only be rebuilt
+// by replaying its sequence); a negative slot marks a padding entry whose outputs
+// are written as zeros and whose state is not touched (as is a slot past the
+// pool's end).
 #include "common.cuh"
 #include "internal.h"
 
@@ -26,7 +46,6 @@ namespace {
 
 template <int CPL> struct vec;
 template <> struct vec<4> {
-  using T = float4;
   static __device__ __forceinline__ void ld(const float *p, float *x) {
     float4 v = __ldcs(reinterpret_cast<const float4 *>(p));
     x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
@@ -47,123 +66,205 @@ template <> struct vec<2> {
 
 constexpr int kWarps = 8;
 
-template <int D_K, int D_V, typename IO, bool CHANNEL_GATE>
+// Per-token row vectors, triple-buffered.
+template <int D_K> struct TokenVecs {
+  float kr[3][D_K];   // recall direction
+  float aq[3][D_K];   // a . q
+  float a[3][D_K];    // decay
+  float e[3][D_K];    // erase coefficient (beta folded in)
+  float bk[3][D_K];   // write coefficient beta k
+  float coef[3][2];   // c_r, c_v = beta k.q
+};
+
+template <int D_K, int D_V, typename IO, bool CHANNEL_GATE, bool DECAY_FIRST>
 __global__ void __launch_bounds__(kWarps * 32, 2)
-decode_step_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
-                   const float *__restrict__ g, const float *__restrict__ beta,
-                   IO *__restrict__ o, float *__restrict__ state, int H_qk, int H_v) {
+recurrent_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
+                 const float *__restrict__ g, const float *__restrict__ beta,
+                 IO *__restrict__ o, float *__restrict__ state,
+                 const int32_t *__restrict__ slots, int64_t num_slots, int T, int H_qk,
+                 int H_v) {
   constexpr int RPW = D_K / kWarps;  // state rows per warp
   constexpr int CPL = D_V / 32;      // state columns per lane
-  static_assert(D_K % (kWarps * 32) == 0 || D_K == 64 || D_K == 128, "d_k");
+  static_assert(D_K == 64 || D_K == 128, "d_k");
 
   const int nh = blockIdx.x;  // n * H_v + h
   const int n = nh / H_v, h = nh - n * H_v;
   const int hk = h / (H_v / H_qk);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  __shared__ float s_k[D_K], s_a[D_K], s_aq[D_K];
-  __shared__ float s_red[2][kWarps][D_V];
-  __shared__ float s_dot[D_K / 32][2];
+  __shared__ TokenVecs<D_K> tv;
+  __shared__ float s_red[2][2][kWarps][D_V];  // [token parity][r | p][warp][column]
+  __shared__ float s_dot[3][D_K / 32][2];     // per-warp k.q, k.(a.q), by token buffer
+
+  const int64_t slot = slots ? (int64_t)__ldg(slots + n) : (int64_t)n;
+  if (slot < 0 || slot >= num_slots) {  // padding entry: zero outputs, state untouched
+    for (int e = threadIdx.x; e < T * D_V; e += kWarps * 32) {
+      const int t = e / D_V, c = e - t * D_V;
+      io<IO>::store(o + (((size_t)n * T + t) * H_v + h) * D_V + c, 0.f);
+    }
+    return;
+  }
 
   // 1. stream this warp's rows of the state into registers (issued first:
-  //    they are >99% of the step's bytes)
-  float *S = state + (size_t)nh * D_K * D_V;
+  //    for a single step they are >99% of the bytes)
+  float *S = state + ((size_t)slot * H_v + h) * D_K * D_V;
   float x[RPW][CPL];
 #pragma unroll
   for (int r = 0; r < RPW; ++r) vec<CPL>::ld(S + (warp * RPW + r) * D_V + lane * CPL, x[r]);
 
-  // 2. the token's key, query and gate (one element per thread)
-  if (threadIdx.x < D_K) {
+  // Token t's inputs: row vectors by threads i < D_K, the value vector and
+  // beta by every thread (the same few bytes, served by L1).
+  auto token_base = [&](int t) { return (size_t)n * T + t; };
+  auto load_raw = [&](int t, float &kk, float &qq, float &gg) {
+    const size_t tok = token_base(t);
     const int i = threadIdx.x;
-    const size_t qk_off = ((size_t)n * H_qk + hk) * D_K + i;
-    const float kk = io<IO>::load(k + qk_off);
-    const float qq = io<IO>::load(q + qk_off);
-    const float gg = CHANNEL_GATE ? __ldg(g + (size_t)nh * D_K + i) : __ldg(g + nh);
+    const size_t qk_off = (tok * H_qk + hk) * D_K + i;
+    kk = io<IO>::load(k + qk_off);
+    qq = io<IO>::load(q + qk_off);
+    gg = CHANNEL_GATE ? __ldg(g + (tok * H_v + h) * D_K + i) : __ldg(g + tok * H_v + h);
+  };
+  auto load_v = [&](int t, float *vv, float &b) {
+    const size_t tok = token_base(t);
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) vv[c] = io<IO>::load(v + (tok * H_v + h) * D_V + lane * CPL + c);
+    b = __ldg(beta + tok * H_v + h);
+  };
+  // Writes token vectors into buffer `buf` (threads i < D_K; warp-uniform).
+  auto stage = [&](int buf, float kk, float qq, float gg, float b) {
+    const int i = threadIdx.x;
     const float a = expf(gg);
-    s_k[i] = kk;
-    s_a[i] = a;
-    s_aq[i] = a * qq;
+    const float aq = a * qq;
+    tv.kr[buf][i] = DECAY_FIRST ? a * kk : kk;
+    tv.aq[buf][i] = aq;
+    tv.a[buf][i] = a;
+    tv.e[buf][i] = DECAY_FIRST ? b * kk : b * a * kk;
+    tv.bk[buf][i] = b * kk;
     const float kq = warp_sum(kk * qq);
-    const float kaq = warp_sum(kk * a * qq);
+    const float kaq = DECAY_FIRST ? 0.f : warp_sum(kk * aq);
     if (lane == 0) {
-      s_dot[i >> 5][0] = kq;
-      s_dot[i >> 5][1] = kaq;
+      s_dot[buf][i >> 5][0] = kq;
+      s_dot[buf][i >> 5][1] = kaq;
+    }
+  };
+
+  float vv[CPL], b;
+  if (T > 0) {
+    load_v(0, vv, b);
+    if (threadIdx.x < D_K) {
+      float kk, qq, gg;
+      load_raw(0, kk, qq, gg);
+      stage(0, kk, qq, gg, b);
     }
   }
-  const float b = __ldg(beta + nh);
-  float vv[CPL];
-#pragma unroll
-  for (int c = 0; c < CPL; ++c) vv[c] = io<IO>::load(v + (size_t)nh * D_V + lane * CPL + c);
   __syncthreads();
-
-  // 3. partial column sums over this warp's rows: r = S^T k, p = S^T (a.q)
-  float rp[CPL], pp[CPL];
-#pragma unroll
-  for (int c = 0; c < CPL; ++c) rp[c] = pp[c] = 0.f;
-#pragma unroll
-  for (int r = 0; r < RPW; ++r) {
-    const float ki = s_k[warp * RPW + r], aqi = s_aq[warp * RPW + r];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      rp[c] = fmaf(ki, x[r][c], rp[c]);
-      pp[c] = fmaf(aqi, x[r][c], pp[c]);
-    }
-  }
-#pragma unroll
-  for (int c = 0; c < CPL; ++c) {
-    s_red[0][warp][lane * CPL + c] = rp[c];
-    s_red[1][warp][lane * CPL + c] = pp[c];
-  }
-  __syncthreads();
-  float rf[CPL];
-#pragma unroll
-  for (int c = 0; c < CPL; ++c) {
-    float acc = 0.f;
-#pragma unroll
-    for (int w = 0; w < kWarps; ++w) acc += s_red[0][w][lane * CPL + c];
-    rf[c] = acc;
-  }
-
-  // 4. S' = a . (S - b k r^T) + b k v^T, written back in place
-#pragma unroll
-  for (int r = 0; r < RPW; ++r) {
-    const int i = warp * RPW + r;
-    const float a = s_a[i], bk = b * s_k[i];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) x[r][c] = fmaf(a, fmaf(-bk, rf[c], x[r][c]), bk * vv[c]);
-    vec<CPL>::st(S + i * D_V + lane * CPL, x[r]);
-  }
-
-  // 5. o = p - b (k.(a.q)) r + b (k.q) v
-  if (warp == 0) {
+  if (threadIdx.x == 0 && T > 0) {
     float kq = 0.f, kaq = 0.f;
 #pragma unroll
     for (int w = 0; w < D_K / 32; ++w) {
-      kq += s_dot[w][0];
-      kaq += s_dot[w][1];
+      kq += s_dot[0][w][0];
+      kaq += s_dot[0][w][1];
+    }
+    tv.coef[0][0] = b * (DECAY_FIRST ? kq : kaq);
+    tv.coef[0][1] = b * kq;
+  }
+
+  for (int t = 0; t < T; ++t) {
+    const int buf = t % 3, par = t & 1;
+    const bool more = t + 1 < T;
+    // prefetch token t+1's inputs into registers
+    float kn = 0.f, qn = 0.f, gn = 0.f, vn[CPL], bn = 0.f;
+    if (more) {
+      load_v(t + 1, vn, bn);
+      if (threadIdx.x < D_K) load_raw(t + 1, kn, qn, gn);
+    }
+
+    // 2. partial column sums over this warp's rows: r = S^T kr, p = S^T (a.q)
+    float rp[CPL], pp[CPL];
+#pragma unroll
+    for (int c = 0; c < CPL; ++c) rp[c] = pp[c] = 0.f;
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const float ki = tv.kr[buf][warp * RPW + r], aqi = tv.aq[buf][warp * RPW + r];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        rp[c] = fmaf(ki, x[r][c], rp[c]);
+        pp[c] = fmaf(aqi, x[r][c], pp[c]);
+      }
     }
 #pragma unroll
     for (int c = 0; c < CPL; ++c) {
-      float p = 0.f;
+      s_red[par][0][warp][lane * CPL + c] = rp[c];
+      s_red[par][1][warp][lane * CPL + c] = pp[c];
+    }
+    // token t+1's vectors go into the buffer token t-2 used (free by now)
+    if (more && threadIdx.x < D_K) stage((t + 1) % 3, kn, qn, gn, bn);
+    __syncthreads();
+
+    float rf[CPL];
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) p += s_red[1][w][lane * CPL + c];
-      const float out = p - b * kaq * rf[c] + b * kq * vv[c];
-      io<IO>::store(o + (size_t)nh * D_V + lane * CPL + c, out);
+    for (int c = 0; c < CPL; ++c) {
+      float acc = 0.f;
+#pragma unroll
+      for (int w = 0; w < kWarps; ++w) acc += s_red[par][0][w][lane * CPL + c];
+      rf[c] = acc;
+    }
+    if (more && threadIdx.x == 32) {  // token t+1's readout coefficients
+      float kq = 0.f, kaq = 0.f;
+#pragma unroll
+      for (int w = 0; w < D_K / 32; ++w) {
+        kq += s_dot[(t + 1) % 3][w][0];
+        kaq += s_dot[(t + 1) % 3][w][1];
+      }
+      tv.coef[(t + 1) % 3][0] = bn * (DECAY_FIRST ? kq : kaq);
+      tv.coef[(t + 1) % 3][1] = bn * kq;
+    }
+
+    // 3. S' = a . S - e r^T + beta k v^T (e folds the order), in registers
+#pragma unroll
+    for (int r = 0; r < RPW; ++r) {
+      const int i = warp * RPW + r;
+      const float a = tv.a[buf][i], e = tv.e[buf][i], bk = tv.bk[buf][i];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) x[r][c] = fmaf(a, x[r][c], fmaf(-e, rf[c], bk * vv[c]));
+    }
+
+    // 4. o = p - c_r r + c_v v
+    if (warp == 0) {
+      const float cr = tv.coef[buf][0], cv = tv.coef[buf][1];
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) {
+        float p = 0.f;
+#pragma unroll
+        for (int w = 0; w < kWarps; ++w) p += s_red[par][1][w][lane * CPL + c];
+        const float out = p - cr * rf[c] + cv * vv[c];
+        io<IO>::store(o + (token_base(t) * H_v + h) * D_V + lane * CPL + c, out);
+      }
+    }
+    if (more) {
+#pragma unroll
+      for (int c = 0; c < CPL; ++c) vv[c] = vn[c];
     }
   }
+
+  // 5. the state goes back once, in place
+#pragma unroll
+  for (int r = 0; r < RPW; ++r) vec<CPL>::st(S + (warp * RPW + r) * D_V + lane * CPL, x[r]);
 }
 
 template <int D_K, int D_V, typename IO>
 cudaError_t launch_dv(const DecodeArgs &a, cudaStream_t s) {
   const unsigned grid = (unsigned)((int64_t)a.N * a.H_v);
-  if (a.channel_gate)
-    decode_step_kernel<D_K, D_V, IO, true><<<grid, kWarps * 32, 0, s>>>(
-        (const IO *)a.q, (const IO *)a.k, (const IO *)a.v, a.g, a.beta, (IO *)a.o, a.state,
-        a.H_qk, a.H_v);
+  const dim3 block(kWarps * 32);
+#define GDR_RECURRENT_ARGS                                                                  \
+  (const IO *)a.q, (const IO *)a.k, (const IO *)a.v, a.g, a.beta, (IO *)a.o, a.state, a.slots, \
+      a.num_slots, a.T, a.H_qk, a.H_v
+  if (!a.channel_gate)
+    recurrent_kernel<D_K, D_V, IO, false, false><<<grid, block, 0, s>>>(GDR_RECURRENT_ARGS);
+  else if (a.decay_first)
+    recurrent_kernel<D_K, D_V, IO, true, true><<<grid, block, 0, s>>>(GDR_RECURRENT_ARGS);
   else
-    decode_step_kernel<D_K, D_V, IO, false><<<grid, kWarps * 32, 0, s>>>(
-        (const IO *)a.q, (const IO *)a.k, (const IO *)a.v, a.g, a.beta, (IO *)a.o, a.state,
-        a.H_qk, a.H_v);
+    recurrent_kernel<D_K, D_V, IO, true, false><<<grid, block, 0, s>>>(GDR_RECURRENT_ARGS);
+#undef GDR_RECURRENT_ARGS
   return cudaGetLastError();
 }
 
@@ -175,13 +276,50 @@ cudaError_t launch_io(const DecodeArgs &a, cudaStream_t s) {
   return launch_dv<64, 64, IO>(a, s);
 }
 
+// dst[dst slot of n] = src[src slot of n] (zeros where the source slot is
+// negative; nothing where the destination slot is negative), one float4 per
+// thread-iteration.  A NULL slot array is the identity.
+__global__ void state_copy_kernel(const float4 *__restrict__ src, const int32_t *__restrict__ src_slots,
+                                  int64_t src_limit, float4 *__restrict__ dst,
+                                  const int32_t *__restrict__ dst_slots, int64_t dst_limit, int N,
+                                  int64_t per_seq4) {
+  const int64_t total = (int64_t)N * per_seq4;
+  for (int64_t idx = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; idx < total;
+       idx += (int64_t)gridDim.x * blockDim.x) {
+    const int n = (int)(idx / per_seq4);
+    const int64_t e = idx - (int64_t)n * per_seq4;
+    const int64_t ds = dst_slots ? (int64_t)__ldg(dst_slots + n) : n;
+    if (ds < 0 || ds >= dst_limit) continue;
+    const int64_t ss = src_slots ? (int64_t)__ldg(src_slots + n) : n;
+    const float4 val = (src && ss >= 0 && ss < src_limit) ? __ldcs(src + ss * per_seq4 + e) : make_float4(0.f, 0.f, 0.f, 0.f);
+    __stcs(dst + ds * per_seq4 + e, val);
+  }
+}
+
 }  // namespace
 
-cudaError_t launch_decode_step(const DecodeArgs &a, cudaStream_t stream) {
+cudaError_t launch_recurrent(const DecodeArgs &a, cudaStream_t stream) {
   if (a.N == 0) return cudaSuccess;
-  TraceScope tr("decode_step_kernel", stream);
+  TraceScope tr("recurrent_kernel", stream);
   if (a.bf16) return launch_io<__nv_bfloat16>(a, stream);
   return launch_io<float>(a, stream);
+}
+
+cudaError_t launch_state_copy(const float *src, const int32_t *src_slots, int64_t src_limit,
+                              float *dst, const int32_t *dst_slots, int64_t dst_limit, int N,
+                              int64_t per_seq_floats, cudaStream_t stream) {
+  if (N == 0 || per_seq_floats == 0) return cudaSuccess;
+  const int64_t per_seq4 = per_seq_floats / 4;
+  const int64_t total = (int64_t)N * per_seq4;
+  const int threads = 256;
+  int64_t blocks = (total + threads - 1) / threads;
+  const int64_t cap = (int64_t)sm_count() * 8;
+  if (blocks > cap) blocks = cap;
+  TraceScope tr("state_copy_kernel", stream);
+  state_copy_kernel<<<(unsigned)blocks, threads, 0, stream>>>(
+      reinterpret_cast<const float4 *>(src), src_slots, src_limit,
+      reinterpret_cast<float4 *>(dst), dst_slots, dst_limit, N, per_seq4);
+  return cudaGetLastError();
 }
 
 }  // namespace gdr

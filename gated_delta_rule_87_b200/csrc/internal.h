@@ -26,17 +26,33 @@ class TraceScope {
 // Sets the text kda_last_error() returns on the calling host thread.
 void set_last_error(const char *msg);
 
+// Multiprocessor count of the current device.
+int sm_count();
+
+// Token-by-token form: T tokens for each of N sequences ([N, T, H, d]
+// layout), state updated in place.  T = 1 is one decode step.
 struct DecodeArgs {
   const void *q, *k, *v;
   const float *g, *beta;
   void *o;
   float *state;
-  int N, H_qk, H_v, d_k, d_v;
+  const int32_t *slots;  // device [N] state-pool slots, or nullptr (slot n = n)
+  int64_t num_slots;     // pool capacity; slots outside [0, num_slots) are padding
+  int N, T, H_qk, H_v, d_k, d_v;
   bool channel_gate;  // KDA (per-channel) or Gated DeltaNet (scalar)
+  bool decay_first;   // decay before the erase (KDA only)
   bool bf16;          // io dtype
 };
 
-cudaError_t launch_decode_step(const DecodeArgs &a, cudaStream_t stream);
+cudaError_t launch_recurrent(const DecodeArgs &a, cudaStream_t stream);
+
+// dst[dst_slots[n]] = src[src_slots[n]] for n < N, per_seq_floats floats per
+// entry (a multiple of 4, 16-byte aligned buffers); NULL slots = identity.
+// A source slot outside [0, src_limit) copies zeros (as does src == NULL); a
+// destination slot outside [0, dst_limit) is skipped.
+cudaError_t launch_state_copy(const float *src, const int32_t *src_slots, int64_t src_limit,
+                              float *dst, const int32_t *dst_slots, int64_t dst_limit, int N,
+                              int64_t per_seq_floats, cudaStream_t stream);
 
 // Chunk length of the prefill kernels (tokens per chunk).
 constexpr int kChunk = 64;
@@ -47,10 +63,13 @@ struct PrefillArgs {
   void *o;
   const float *initial_state;
   float *final_state;
+  const int32_t *state_slots;  // device [num_seqs] pool slots of the states, or nullptr
+  int64_t num_slots;           // pool capacity (slots outside [0, num_slots): no state)
   const int32_t *cu_seqlens;  // device, or nullptr (dense)
   int num_seqs;               // N
   int B, T, H_qk, H_v, d_k, d_v;
   bool channel_gate;
+  bool decay_first;  // decay before the erase (KDA only)
   bool bf16;
   // workspace (device); status word at offset 0
   void *workspace;

@@ -22,6 +22,11 @@
 // difference that is <= 0, so no factor exceeds 1 and no range limit applies
 // to g.
 //
+// With the decay applied before the erase (DECAY_FIRST, the variant order
+// (I - beta k k^T) Diag(a) S), recall reads the state along a_t . k_t, so the
+// erase direction equals the write direction: every Gp above becomes G, and
+// the rest of the computation is unchanged.
+//
 // Mapping: one CTA per (sequence, v-head, slice of NS state columns); the
 // CTA walks its sequence's chunks in order with the state slice in shared
 // memory.  The d_v columns of the state evolve independently (the update
@@ -53,13 +58,14 @@ struct SimtSmem {
   float beta[C];
 };
 
-template <int D_K, int D_V, typename IO, bool CHANNEL_GATE>
+template <int D_K, int D_V, typename IO, bool CHANNEL_GATE, bool DECAY_FIRST>
 __global__ void __launch_bounds__(kThreads, 1)
 prefill_simt_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
                     const float *__restrict__ g, const float *__restrict__ beta,
-                    IO *__restrict__ o, const float *__restrict__ s0, float *__restrict__ sT,
-                    const int32_t *__restrict__ cu, int T, int H_qk, int H_v,
-                    const int32_t *__restrict__ status) {
+                    IO *__restrict__ o, const float *s0, float *sT,
+                    const int32_t *__restrict__ state_slots, int64_t num_slots,
+                    const int32_t *__restrict__ cu,
+                    int T, int H_qk, int H_v, const int32_t *__restrict__ status) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   using Sm = SimtSmem<D_K>;
   Sm &sm = *reinterpret_cast<Sm *>(smem_raw);
@@ -83,8 +89,13 @@ prefill_simt_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO
     eos = bos + T;
   }
 
-  // initial state slice
-  const size_t state_off = ((size_t)n * H_v + h) * D_K * D_V;
+  // initial state slice (a negative pool slot: zeros in, nothing out)
+  const int64_t slot = state_slots ? (int64_t)state_slots[n] : (int64_t)n;
+  if (slot < 0 || slot >= num_slots) {
+    s0 = nullptr;
+    sT = nullptr;
+  }
+  const size_t state_off = ((size_t)slot * H_v + h) * D_K * D_V;
   for (int e = tid; e < D_K * NS; e += kThreads) {
     const int i = e / NS, j = e % NS;
     sm.S[i][j] = s0 ? s0[state_off + (size_t)i * D_V + col0 + j] : 0.f;
@@ -132,8 +143,8 @@ prefill_simt_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO
       float aw = 0.f, ae = 0.f, bw = 0.f, be = 0.f;
       if (j <= i) {
         for (int c = 0; c < D_K; ++c) {
-          const float Gi = sm.G[i][c], Gpi = (i > 0) ? sm.G[i - 1][c] : 0.f;
-          const float Gj = sm.G[j][c], Gpj = (j > 0) ? sm.G[j - 1][c] : 0.f;
+          const float Gi = sm.G[i][c], Gpi = DECAY_FIRST ? Gi : (i > 0) ? sm.G[i - 1][c] : 0.f;
+          const float Gj = sm.G[j][c], Gpj = DECAY_FIRST ? Gj : (j > 0) ? sm.G[j - 1][c] : 0.f;
           const float kj = sm.K[j][c];
           const float qk = sm.Q[i][c] * kj;
           bw = fmaf(qk, expf(Gi - Gj), bw);
@@ -176,7 +187,7 @@ prefill_simt_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO
       const int i = e / NS, j = e % NS;
       float acc = 0.f;
       for (int c = 0; c < D_K; ++c) {
-        const float Gpi = (i > 0) ? sm.G[i - 1][c] : 0.f;
+        const float Gpi = DECAY_FIRST ? sm.G[i][c] : (i > 0) ? sm.G[i - 1][c] : 0.f;
         acc = fmaf(sm.K[i][c] * expf(Gpi), sm.S[c][j], acc);
       }
       for (int jj = 0; jj < i; ++jj) acc = fmaf(sm.Aw[i][jj] * sm.beta[jj], sm.V[jj][j], acc);
@@ -209,7 +220,7 @@ prefill_simt_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO
       const float GL = sm.G[C - 1][c];  // rows >= L carry g = 0, so this is G_L
       float acc = expf(GL) * sm.S[c][j];
       for (int t = 0; t < L; ++t) {
-        const float Gt = sm.G[t][c], Gpt = (t > 0) ? sm.G[t - 1][c] : 0.f;
+        const float Gt = sm.G[t][c], Gpt = DECAY_FIRST ? Gt : (t > 0) ? sm.G[t - 1][c] : 0.f;
         const float bk = sm.beta[t] * sm.K[t][c];
         acc = fmaf(bk * expf(GL - Gt), sm.V[t][j], acc);
         acc = fmaf(-bk * expf(GL - Gpt), sm.R[t][j], acc);
@@ -228,7 +239,8 @@ prefill_simt_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO
 
 template <int D_K, int D_V, typename IO, bool CG>
 cudaError_t launch_cfg(const PrefillArgs &a, cudaStream_t s) {
-  auto kern = prefill_simt_kernel<D_K, D_V, IO, CG>;
+  auto kern = (CG && a.decay_first) ? prefill_simt_kernel<D_K, D_V, IO, CG, true>
+                                    : prefill_simt_kernel<D_K, D_V, IO, CG, false>;
   const int smem = (int)sizeof(SimtSmem<D_K>);
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -237,7 +249,7 @@ cudaError_t launch_cfg(const PrefillArgs &a, cudaStream_t s) {
   TraceScope tr("prefill_simt_kernel", s);
   kern<<<grid, kThreads, smem, s>>>((const IO *)a.q, (const IO *)a.k, (const IO *)a.v, a.g,
                                    a.beta, (IO *)a.o, a.initial_state, a.final_state,
-                                   a.cu_seqlens, a.T, a.H_qk, a.H_v,
+                                   a.state_slots, a.num_slots, a.cu_seqlens, a.T, a.H_qk, a.H_v,
                                    (const int32_t *)a.workspace);
   return cudaGetLastError();
 }

@@ -28,18 +28,26 @@
 // sub-chunks and at most e^{16 |g|max} inside the diagonal sub-chunk, which
 // stays in fp32/bf16 range for per-token log-decays g >= -5.
 //
+// With the decay applied before the erase (the variant order (I - beta k
+// k^T) Diag(a) S), recall reads the state along a_t . k_t: the erase
+// direction equals the write direction, every Gp above becomes G, and only
+// the operand scale factors change (template flag DECAY_FIRST).
+//
 // Two kernels (plus a one-CTA planning kernel):
-//   prep  -- one CTA per (chunk, v-head), all chunks in parallel: loads
-//            q/k/v/g tiles with TMA, builds every S-independent factor above
-//            with tcgen05 MMAs (bf16 operands, fp32 accumulators in TMEM) and
-//            a blocked fp32 triangular inverse, and writes P, Q', Qc,
-//            O_intra (bf16) into a workspace slot laid out as the scan's
-//            shared-memory operand images.
-//   scan  -- one CTA per (sequence, v-head, 32-column slice of the state),
-//            walks the chunks in order with the fp32 state slice in
-//            registers: one MMA P S (128x32x128) and one Q' S (64x32x128)
-//            per chunk, then S <- P S + Qc and o = Q' S + O_intra.  The
-//            state columns evolve independently, so slices never talk.
+//   prep  -- persistent, one CTA per SM looping over (chunk, v-head) items,
+//            all chunks in parallel: loads q/k/v/g tiles with TMA (the next
+//            item's loads overlap the current item's last products), builds
+//            every S-independent factor above with tcgen05 MMAs (bf16
+//            operands, fp32 accumulators in TMEM) and a blocked fp32
+//            triangular inverse, and writes P, Q', Qc, O_intra (bf16) into a
+//            workspace slot laid out as the scan's shared-memory operand
+//            images.
+//   scan  -- one CTA per (sequence, v-head), walking the chunks in order
+//            with the fp32 state in registers of 8 chain warps and its bf16
+//            transpose in TMEM as the A operand: per chunk one MMA
+//            (P S)^T = S^T P^T (128x128x128) and one o^T = S^T Q'^T
+//            (128x64x128), then S <- P S + Qc and o = Q' S + O_intra, with a
+//            load warp double-buffering the slots and 4 output warps.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -225,7 +233,7 @@ __device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
 
 __device__ __forceinline__ void st16(unsigned char *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
 
-template <bool CHANNEL>
+template <bool CHANNEL, bool DECAY_FIRST>
 __global__ void __launch_bounds__(kPrepThreads, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
@@ -419,10 +427,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float k0 = ok ? bf16_lo(kraw) : 0.f, k1 = ok ? bf16_hi(kraw) : 0.f;
       const float q0 = ok ? bf16_lo(qraw) : 0.f, q1 = ok ? bf16_hi(qraw) : 0.f;
       const float b = sBeta[t];
-      const float bk0 = pq0, bk1 = pq1;                       // e^{Gp_t - E_{I-1}}
       const float bq0 = pq0 * a0[r], bq1 = pq1 * a1[r];       // e^{G_t - E_{I-1}}
+      const float bk0 = DECAY_FIRST ? bq0 : pq0;              // e^{Gp_t - E_{I-1}}
+      const float bk1 = DECAY_FIRST ? bq1 : pq1;
       const float rw0 = w0[r], rw1 = w1[r];                   // e^{E_I - G_t}
-      const float re0 = rw0 * a0[r], re1 = rw1 * a1[r];       // e^{E_I - Gp_t}
+      const float re0 = DECAY_FIRST ? rw0 : rw0 * a0[r];      // e^{E_I - Gp_t}
+      const float re1 = DECAY_FIRST ? rw1 : rw1 * a1[r];
       pq0 = bq0;
       pq1 = bq1;
       const int rowK = 32 * bI + 8 * rh + r, rowQ = rowK + 16;
@@ -833,8 +843,9 @@ constexpr int kOutBarrier = 1;   // named barrier among the output warps
 __global__ void __launch_bounds__(kScanThreads, 1)
 chunk_scan_kernel(const int32_t *hdr, const int32_t *__restrict__ seq_off,
                   const ChunkEntry *__restrict__ tab, const unsigned char *__restrict__ slots,
-                  __nv_bfloat16 *__restrict__ o, const float *__restrict__ s0,
-                  float *__restrict__ sT, int H_v, int32_t *err) {
+                  __nv_bfloat16 *__restrict__ o, const float *s0, float *sT,
+                  const int32_t *__restrict__ state_slots, int64_t num_slots, int H_v,
+                  int32_t *err) {
   extern __shared__ unsigned char smem_raw[];
   // 1024-byte aligned base, derived by pointer arithmetic on the shared array so
   // that the compiler keeps shared-memory addressing for every access
@@ -874,7 +885,13 @@ chunk_scan_kernel(const int32_t *hdr, const int32_t *__restrict__ seq_off,
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tslot;
-  const size_t state_base = ((size_t)n * H_v + h) * DK * DK;
+  // the state's pool slot; a negative slot starts from zeros and keeps no final state
+  const int64_t sslot = state_slots ? (int64_t)state_slots[n] : (int64_t)n;
+  if (sslot < 0 || sslot >= num_slots) {
+    s0 = nullptr;
+    sT = nullptr;
+  }
+  const size_t state_base = ((size_t)sslot * H_v + h) * DK * DK;
 
   if (warp == kLoadWarp) {
     // ---------------- loads ----------------
@@ -1032,13 +1049,6 @@ chunk_scan_kernel(const int32_t *hdr, const int32_t *__restrict__ seq_off,
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
-int sm_count() {
-  int dev = 0, n = 148;
-  if (cudaGetDevice(&dev) == cudaSuccess)
-    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
-  return n > 0 ? n : 148;
-}
-
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   static std::once_flag once;
@@ -1111,7 +1121,9 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  auto prep = a.channel_gate ? chunk_prep_kernel<true> : chunk_prep_kernel<false>;
+  auto prep = !a.channel_gate ? chunk_prep_kernel<false, false>
+               : a.decay_first ? chunk_prep_kernel<true, true>
+                               : chunk_prep_kernel<true, false>;
   e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM);
   if (e != cudaSuccess) return e;
   const int64_t items = max_chunks * a.H_v;
@@ -1130,7 +1142,8 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
   {
     TraceScope tr("chunk_scan_kernel", stream);
     chunk_scan_kernel<<<gs, kScanThreads, SCAN_SMEM, stream>>>(
-        hdr, seq_off, tab, slots, (__nv_bfloat16 *)a.o, a.initial_state, a.final_state, a.H_v, hdr);
+        hdr, seq_off, tab, slots, (__nv_bfloat16 *)a.o, a.initial_state, a.final_state,
+        a.state_slots, a.num_slots, a.H_v, hdr);
   }
   return cudaGetLastError();
 }

@@ -69,6 +69,18 @@ typedef enum {
 
 typedef enum { KDA_F32 = 0, KDA_BF16 = 1 } kda_dtype_t;
 
+/* Where the per-channel decay sits relative to the rank-one erase (KDA only;
+ * for a scalar gate the two orders are the same operator).
+ *   KDA_ERASE_THEN_DECAY  S_t = Diag(a_t)(I - beta_t k_t k_t^T) S_{t-1} + beta_t k_t v_t^T
+ *                         the operator as the table row "KDA" writes it (default);
+ *   KDA_DECAY_THEN_ERASE  S_t = (I - beta_t k_t k_t^T) Diag(a_t) S_{t-1} + beta_t k_t v_t^T
+ *                         the erase acts on the decayed state, so that with
+ *                         beta = 1 and |k| = 1 the update writes only the
+ *                         difference between v and what the decayed memory
+ *                         recalls (ai-explained.dataextractor.workers.dev
+ *                         "The efficiency lineage", item 8 "Delta rule"). */
+typedef enum { KDA_ERASE_THEN_DECAY = 0, KDA_DECAY_THEN_ERASE = 1 } kda_order_t;
+
 /* Device-side error codes written to the workspace status word. */
 #define KDA_DEVICE_OK 0
 #define KDA_DEVICE_BAD_CU_SEQLENS 1  /* cu[0] != 0, decreasing, or cu[N] != T */
@@ -149,6 +161,101 @@ KDA_API kda_status_t gdn_decode_step(const void *q, const void *k, const void *v
                              const float *beta, void *o, float *state, int32_t N,
                              int32_t H_qk, int32_t H_v, int32_t d_k, int32_t d_v,
                              kda_dtype_t io_dtype, void *stream);
+
+/* --------------------------------------------------------------------------
+ * Prefill with the decay order and a state pool (KDA and Gated DeltaNet).
+ * Same operation, arguments and errors as kda_chunk_fwd / gdn_chunk_fwd, plus:
+ *
+ *   order        KDA_ERASE_THEN_DECAY (what kda_chunk_fwd computes) or
+ *                KDA_DECAY_THEN_ERASE; gdn has no order argument.
+ *   state_slots  int32 DEVICE array [N] (N = B, or num_seqs with cu_seqlens),
+ *                or NULL.  When given, initial_state and final_state are
+ *                POOLS of num_slots states [num_slots, H, d_k, d_v] and
+ *                sequence n reads its initial state from slot state_slots[n]
+ *                and writes its final state to the same slot.  initial_state
+ *                and final_state may be the same pool (in-place update of a
+ *                serving state pool: inferencex.semianalysis.com "Linear
+ *                attention", "Why it matters": a dropped state can only be
+ *                rebuilt by replaying the sequence, so it is checkpointed).
+ *                A slot outside [0, num_slots) means "no slot": the sequence
+ *                starts from zeros and its final state is not stored.  Two
+ *                sequences must not share a slot (the slot's contents are
+ *                then unspecified).
+ *   num_slots    pool capacity (ignored when state_slots is NULL).
+ * ------------------------------------------------------------------------ */
+KDA_API kda_status_t kda_chunk_fwd_ex(const void *q, const void *k, const void *v,
+                                      const float *g, const float *beta, void *o,
+                                      const float *initial_state, float *final_state,
+                                      const int32_t *state_slots, int64_t num_slots,
+                                      const int32_t *cu_seqlens, int32_t num_seqs, int32_t B,
+                                      int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                      kda_order_t order, kda_dtype_t io_dtype, void *workspace,
+                                      size_t workspace_bytes, void *stream);
+
+KDA_API kda_status_t gdn_chunk_fwd_ex(const void *q, const void *k, const void *v,
+                                      const float *g, const float *beta, void *o,
+                                      const float *initial_state, float *final_state,
+                                      const int32_t *state_slots, int64_t num_slots,
+                                      const int32_t *cu_seqlens, int32_t num_seqs, int32_t B,
+                                      int32_t T, int32_t H_qk, int32_t H_v, int32_t d_k,
+                                      int32_t d_v, kda_dtype_t io_dtype, void *workspace,
+                                      size_t workspace_bytes, void *stream);
+
+/* --------------------------------------------------------------------------
+ * Token-by-token form for a few tokens per sequence: T consecutive tokens of
+ * each of N sequences (T = 1 is one decode step; T > 1 serves speculative
+ * decoding or a prompt fed in small pieces), applied one after another to
+ * the state, which is read from HBM once and written back once, in place.
+ * The result equals T single decode steps (and a prefill of the same tokens).
+ *
+ *   q, k  [N, T, H_qk, d_k] io_dtype;  v, o [N, T, H_v, d_v] io_dtype
+ *   g     [N, T, H_v, d_k] fp32 (KDA) or [N, T, H_v] fp32 (GDN)
+ *   beta  [N, T, H_v] fp32
+ *   state the states, [N, H_v, d_k, d_v] fp32 when state_slots is NULL; else
+ *         a pool [num_slots, H_v, d_k, d_v] of which sequence n uses slot
+ *         state_slots[n] (int32 DEVICE array [N]).  A slot outside
+ *         [0, num_slots) marks a padding entry: its o rows are written as
+ *         zeros and no state is touched.  Slots of different sequences must
+ *         differ.
+ *   order KDA only, as in kda_chunk_fwd_ex.
+ * Alignment as the decode step; state_slots 4-byte aligned.  No workspace.
+ * Any T >= 0 is accepted; past a chunk's worth of tokens the chunked prefill
+ * is the faster route.
+ * ------------------------------------------------------------------------ */
+KDA_API kda_status_t kda_recurrent_fwd(const void *q, const void *k, const void *v,
+                                       const float *g, const float *beta, void *o, float *state,
+                                       const int32_t *state_slots, int64_t num_slots, int32_t N,
+                                       int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                       kda_order_t order, kda_dtype_t io_dtype, void *stream);
+
+KDA_API kda_status_t gdn_recurrent_fwd(const void *q, const void *k, const void *v,
+                                       const float *g, const float *beta, void *o, float *state,
+                                       const int32_t *state_slots, int64_t num_slots, int32_t N,
+                                       int32_t T, int32_t H_qk, int32_t H_v, int32_t d_k,
+                                       int32_t d_v, kda_dtype_t io_dtype, void *stream);
+
+/* --------------------------------------------------------------------------
+ * State checkpoint / transfer for a serving state pool
+ * (inferencex.semianalysis.com "Linear attention", "How to read it in
+ * InferenceX": engines checkpoint and transfer the recurrent state so that a
+ * repeated turn does not pay its prefill again).  Batched copies of whole states [H, d_k, d_v] fp32 by slot:
+ *
+ *   kda_state_gather   out[n]  = pool[state_slots[n]]   (zeros for a slot
+ *                                                        outside [0, num_slots))
+ *   kda_state_scatter  pool[state_slots[n]] = src[n]    (skipped for a slot
+ *                                                        outside [0, num_slots))
+ *
+ * pool is [num_slots, H, d_k, d_v]; out/src are dense [N, H, d_k, d_v]; all
+ * DEVICE pointers, 16-byte aligned, pool and dense buffer distinct; slots
+ * int32 DEVICE [N], non-NULL.  Scatter slots must be distinct.  For a copy
+ * to or from host memory, gather into a dense device buffer first.
+ * ------------------------------------------------------------------------ */
+KDA_API kda_status_t kda_state_gather(const float *pool, const int32_t *state_slots,
+                                      int64_t num_slots, float *out, int32_t N, int32_t H,
+                                      int32_t d_k, int32_t d_v, void *stream);
+KDA_API kda_status_t kda_state_scatter(const float *src, float *pool,
+                                       const int32_t *state_slots, int64_t num_slots, int32_t N,
+                                       int32_t H, int32_t d_k, int32_t d_v, void *stream);
 
 /* --------------------------------------------------------------------------
  * kda_chunk_fwd for callers that cannot allocate device memory (the pages

@@ -102,3 +102,72 @@ def test_binding_has_no_cpu_path():
     """The product binding never imports the oracle."""
     src = open(os.path.join(ROOT, "gated_delta_rule_87_b200", "__init__.py")).read()
     assert "oracle" not in re.sub(r'""".*?"""', "", src, flags=re.S)
+
+
+def _prefill_ex(order=0, slots=None, num_slots=0, **over):
+    L = gdr.lib()
+    kw = dict(q=FAKE, k=FAKE, v=FAKE, g=FAKE, beta=FAKE, o=FAKE + 4096, ws=FAKE, ws_bytes=1 << 20)
+    kw.update(over)
+    return L.kda_chunk_fwd_ex(kw["q"], kw["k"], kw["v"], kw["g"], kw["beta"], kw["o"], None, None,
+                              slots, num_slots, None, 0, 1, 64, 2, 128, 128, order, 1, kw["ws"],
+                              kw["ws_bytes"], None)
+
+
+@pytest.mark.parametrize("kw", [
+    dict(order=2), dict(order=-1),                  # no such decay order
+    dict(slots=FAKE + 2, num_slots=4),              # misaligned slot array
+    dict(slots=FAKE, num_slots=-1),                 # negative pool size
+])
+def test_prefill_ex_rejects_bad_arguments_on_host(kw):
+    assert _prefill_ex(**kw) == gdr.KDA_ERR_INVALID_ARG
+    assert gdr.lib().kda_last_error()
+
+
+def _recurrent(order=0, slots=None, num_slots=0, N=4, T=3, ptr=FAKE, o=FAKE + 8192):
+    L = gdr.lib()
+    return L.kda_recurrent_fwd(ptr, FAKE, FAKE, FAKE, FAKE, o, FAKE + 16384, slots, num_slots,
+                               N, T, 2, 128, 128, order, 1, None)
+
+
+@pytest.mark.parametrize("kw,status", [
+    (dict(order=5), gdr.KDA_ERR_INVALID_ARG),
+    (dict(slots=FAKE + 1, num_slots=3), gdr.KDA_ERR_INVALID_ARG),
+    (dict(slots=FAKE, num_slots=-3), gdr.KDA_ERR_INVALID_ARG),
+    (dict(T=-1), gdr.KDA_ERR_INVALID_ARG),
+    (dict(ptr=None), gdr.KDA_ERR_INVALID_ARG),
+    (dict(o=FAKE), gdr.KDA_ERR_INVALID_ARG),        # o aliases q
+])
+def test_recurrent_rejects_bad_arguments_on_host(kw, status):
+    assert _recurrent(**kw) == status
+
+
+def test_recurrent_without_tokens_launches_nothing():
+    """N = 0 or T = 0 returns before any CUDA call (works without a GPU)."""
+    assert _recurrent(N=0, ptr=None) == gdr.KDA_OK
+    assert _recurrent(T=0, ptr=None) == gdr.KDA_OK
+
+
+def test_gdn_recurrent_rejects_indivisible_head_groups():
+    L = gdr.lib()
+    st = L.gdn_recurrent_fwd(FAKE, FAKE, FAKE, FAKE, FAKE, FAKE + 8192, FAKE + 16384, None, 0,
+                             4, 2, 3, 4, 128, 128, 1, None)
+    assert st == gdr.KDA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("args,status", [
+    ((FAKE, None, 8, FAKE + 4096, 4, 2, 128, 128), gdr.KDA_ERR_INVALID_ARG),   # no slots
+    ((FAKE, FAKE, 8, FAKE, 4, 2, 128, 128), gdr.KDA_ERR_INVALID_ARG),          # pool == out
+    ((FAKE + 4, FAKE, 8, FAKE + 4096, 4, 2, 128, 128), gdr.KDA_ERR_INVALID_ARG),  # misaligned
+    ((FAKE, FAKE, -1, FAKE + 4096, 4, 2, 128, 128), gdr.KDA_ERR_INVALID_ARG),  # negative pool
+    ((FAKE, FAKE, 8, FAKE + 4096, 4, 2, 96, 128), gdr.KDA_ERR_UNSUPPORTED),
+    ((None, None, 0, None, 0, 2, 128, 128), gdr.KDA_OK),                       # nothing to copy
+])
+def test_state_gather_validation(args, status):
+    assert gdr.lib().kda_state_gather(*args, None) == status
+
+
+def test_state_scatter_validation():
+    L = gdr.lib()
+    assert L.kda_state_scatter(FAKE, FAKE + 4096, None, 8, 4, 2, 128, 128, None) == \
+        gdr.KDA_ERR_INVALID_ARG
+    assert L.kda_state_scatter(None, None, None, 0, 0, 2, 128, 128, None) == gdr.KDA_OK
