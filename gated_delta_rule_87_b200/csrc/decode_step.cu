@@ -27,10 +27,13 @@
 // [l*D_V/32, (l+1)*D_V/32), loaded with one 16-byte (d_v = 128) or 8-byte
 // (d_v = 64) streaming load per row, so every warp load is a contiguous
 // 512-byte (256-byte) row.  The column sums r and p are reduced over the
-// rows of a warp in registers and across warps through shared memory.  Per
-// token there is one block barrier: the per-token vectors are triple-buffered
-// and the cross-warp partial sums double-buffered, so the next token's
-// vectors are written while the current token is still being applied.
+// rows of a warp in registers and across warps through shared memory; each
+// warp then writes the readout of its own slice of the columns.  Tokens are
+// taken in blocks of 8: one warp per token stages its vectors (decay,
+// recall and erase directions, the readout coefficients) into shared memory
+// while L2 is asked for the next block's rows, so the per-token chain has one
+// block barrier and no global-memory round trip; the cross-warp partial sums
+// are double-buffered by token parity.
 //
 // State pool: with a slot array the state of sequence n is pool[slots[n]]
 // (checkpointed recurrent states for serving, inferencex.semianalysis.com
@@ -46,6 +49,13 @@ namespace {
 
 template <int CPL> struct vec;
 template <> struct vec<4> {
+  static __device__ __forceinline__ void sts(float *p, const float *x) {
+    *reinterpret_cast<float4 *>(p) = make_float4(x[0], x[1], x[2], x[3]);
+  }
+  static __device__ __forceinline__ void lds(const float *p, float *x) {
+    const float4 v = *reinterpret_cast<const float4 *>(p);
+    x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
+  }
   static __device__ __forceinline__ void ld(const float *p, float *x) {
     float4 v = __ldcs(reinterpret_cast<const float4 *>(p));
     x[0] = v.x; x[1] = v.y; x[2] = v.z; x[3] = v.w;
@@ -55,6 +65,13 @@ template <> struct vec<4> {
   }
 };
 template <> struct vec<2> {
+  static __device__ __forceinline__ void sts(float *p, const float *x) {
+    *reinterpret_cast<float2 *>(p) = make_float2(x[0], x[1]);
+  }
+  static __device__ __forceinline__ void lds(const float *p, float *x) {
+    const float2 v = *reinterpret_cast<const float2 *>(p);
+    x[0] = v.x; x[1] = v.y;
+  }
   static __device__ __forceinline__ void ld(const float *p, float *x) {
     float2 v = __ldcs(reinterpret_cast<const float2 *>(p));
     x[0] = v.x; x[1] = v.y;
@@ -66,25 +83,37 @@ template <> struct vec<2> {
 
 constexpr int kWarps = 8;
 
-// Per-token row vectors, triple-buffered.
-template <int D_K> struct TokenVecs {
-  float kr[3][D_K];   // recall direction
-  float aq[3][D_K];   // a . q
-  float a[3][D_K];    // decay
-  float e[3][D_K];    // erase coefficient (beta folded in)
-  float bk[3][D_K];   // write coefficient beta k
-  float coef[3][2];   // c_r, c_v = beta k.q
+// Per-token vectors of a block of up to TB tokens, staged one warp per token.
+template <int D_K, int D_V, int TB> struct BlockVecs {
+  float kr[TB][D_K];   // recall direction
+  float aq[TB][D_K];   // a . q
+  float a[TB][D_K];    // decay
+  float e[TB][D_K];    // erase coefficient (beta folded in)
+  float bk[TB][D_K];   // write coefficient beta k
+  float v[TB][D_V];    // value
+  float coef[TB][2];   // c_r, c_v = beta k.q
 };
 
-template <int D_K, int D_V, typename IO, bool CHANNEL_GATE, bool DECAY_FIRST>
+__device__ __forceinline__ void prefetch_l2(const void *p) {
+  asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+}
+
+// SINGLE: exactly one token (a decode step), known at compile time, so each
+// state row goes back to HBM as soon as it is updated.
+template <int D_K, int D_V, typename IO, bool CHANNEL_GATE, bool DECAY_FIRST, bool SINGLE>
 __global__ void __launch_bounds__(kWarps * 32, 2)
 recurrent_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *__restrict__ v,
                  const float *__restrict__ g, const float *__restrict__ beta,
                  IO *__restrict__ o, float *__restrict__ state,
-                 const int32_t *__restrict__ slots, int64_t num_slots, int T, int H_qk,
+                 const int32_t *__restrict__ slots, int64_t num_slots, int T_arg, int H_qk,
                  int H_v) {
-  constexpr int RPW = D_K / kWarps;  // state rows per warp
-  constexpr int CPL = D_V / 32;      // state columns per lane
+  const int T = SINGLE ? 1 : T_arg;
+  constexpr int TB = SINGLE ? 1 : kWarps;  // tokens per staged block
+  constexpr int RPW = D_K / kWarps;        // state rows per warp
+  constexpr int CPL = D_V / 32;            // state columns per lane
+  // readout: warp w writes columns [w*CW, (w+1)*CW); NP lanes share a column,
+  // each summing the partials of WPP warps
+  constexpr int CW = D_V / kWarps, NP = 32 / CW, WPP = kWarps / NP;
   static_assert(D_K == 64 || D_K == 128, "d_k");
 
   const int nh = blockIdx.x;  // n * H_v + h
@@ -92,9 +121,8 @@ recurrent_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *_
   const int hk = h / (H_v / H_qk);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
 
-  __shared__ TokenVecs<D_K> tv;
-  __shared__ float s_red[2][2][kWarps][D_V];  // [token parity][r | p][warp][column]
-  __shared__ float s_dot[3][D_K / 32][2];     // per-warp k.q, k.(a.q), by token buffer
+  __shared__ __align__(16) BlockVecs<D_K, D_V, TB> bv;
+  __shared__ __align__(16) float s_red[2][2][kWarps][D_V];  // [token parity][r | p][warp][column]
 
   const int64_t slot = slots ? (int64_t)__ldg(slots + n) : (int64_t)n;
   if (slot < 0 || slot >= num_slots) {  // padding entry: zero outputs, state untouched
@@ -112,143 +140,124 @@ recurrent_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *_
 #pragma unroll
   for (int r = 0; r < RPW; ++r) vec<CPL>::ld(S + (warp * RPW + r) * D_V + lane * CPL, x[r]);
 
-  // Token t's inputs: row vectors by threads i < D_K, the value vector and
-  // beta by every thread (the same few bytes, served by L1).
   auto token_base = [&](int t) { return (size_t)n * T + t; };
-  auto load_raw = [&](int t, float &kk, float &qq, float &gg) {
+  // One warp stages token t into block entry tt: the row vectors, the value
+  // and the readout coefficients (k.q and k.(a.q) by a warp reduction).
+  auto stage = [&](int tt, int t) {
     const size_t tok = token_base(t);
-    const int i = threadIdx.x;
-    const size_t qk_off = (tok * H_qk + hk) * D_K + i;
-    kk = io<IO>::load(k + qk_off);
-    qq = io<IO>::load(q + qk_off);
-    gg = CHANNEL_GATE ? __ldg(g + (tok * H_v + h) * D_K + i) : __ldg(g + tok * H_v + h);
-  };
-  auto load_v = [&](int t, float *vv, float &b) {
-    const size_t tok = token_base(t);
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) vv[c] = io<IO>::load(v + (tok * H_v + h) * D_V + lane * CPL + c);
-    b = __ldg(beta + tok * H_v + h);
-  };
-  // Writes token vectors into buffer `buf` (threads i < D_K; warp-uniform).
-  auto stage = [&](int buf, float kk, float qq, float gg, float b) {
-    const int i = threadIdx.x;
-    const float a = expf(gg);
-    const float aq = a * qq;
-    tv.kr[buf][i] = DECAY_FIRST ? a * kk : kk;
-    tv.aq[buf][i] = aq;
-    tv.a[buf][i] = a;
-    tv.e[buf][i] = DECAY_FIRST ? b * kk : b * a * kk;
-    tv.bk[buf][i] = b * kk;
-    const float kq = warp_sum(kk * qq);
-    const float kaq = DECAY_FIRST ? 0.f : warp_sum(kk * aq);
-    if (lane == 0) {
-      s_dot[buf][i >> 5][0] = kq;
-      s_dot[buf][i >> 5][1] = kaq;
-    }
-  };
-
-  float vv[CPL], b;
-  if (T > 0) {
-    load_v(0, vv, b);
-    if (threadIdx.x < D_K) {
-      float kk, qq, gg;
-      load_raw(0, kk, qq, gg);
-      stage(0, kk, qq, gg, b);
-    }
-  }
-  __syncthreads();
-  if (threadIdx.x == 0 && T > 0) {
+    const float b = __ldg(beta + tok * H_v + h);
+    const float gsc = CHANNEL_GATE ? 0.f : __ldg(g + tok * H_v + h);
     float kq = 0.f, kaq = 0.f;
 #pragma unroll
-    for (int w = 0; w < D_K / 32; ++w) {
-      kq += s_dot[0][w][0];
-      kaq += s_dot[0][w][1];
+    for (int j = 0; j < D_K / 32; ++j) {
+      const int i = lane + 32 * j;
+      const size_t qk_off = (tok * H_qk + hk) * D_K + i;
+      const float kk = io<IO>::load(k + qk_off), qq = io<IO>::load(q + qk_off);
+      const float a = expf(CHANNEL_GATE ? __ldg(g + (tok * H_v + h) * D_K + i) : gsc);
+      const float aq = a * qq;
+      bv.kr[tt][i] = DECAY_FIRST ? a * kk : kk;
+      bv.aq[tt][i] = aq;
+      bv.a[tt][i] = a;
+      bv.e[tt][i] = DECAY_FIRST ? b * kk : b * a * kk;
+      bv.bk[tt][i] = b * kk;
+      kq = fmaf(kk, qq, kq);
+      kaq = fmaf(kk, aq, kaq);
     }
-    tv.coef[0][0] = b * (DECAY_FIRST ? kq : kaq);
-    tv.coef[0][1] = b * kq;
-  }
+#pragma unroll
+    for (int j = 0; j < D_V / 32; ++j)
+      bv.v[tt][lane + 32 * j] = io<IO>::load(v + (tok * H_v + h) * D_V + lane + 32 * j);
+    kq = warp_sum(kq);
+    kaq = DECAY_FIRST ? 0.f : warp_sum(kaq);
+    if (lane == 0) {
+      bv.coef[tt][0] = b * (DECAY_FIRST ? kq : kaq);
+      bv.coef[tt][1] = b * kq;
+    }
+  };
+  // One warp asks L2 for token t's input rows (128-byte lines).
+  auto prefetch_token = [&](int t) {
+    const size_t tok = token_base(t);
+    auto rows = [&](const void *p, int bytes) {
+      for (int off = lane * 128; off < bytes; off += 32 * 128)
+        prefetch_l2(static_cast<const char *>(p) + off);
+    };
+    rows(k + (tok * H_qk + hk) * D_K, D_K * (int)sizeof(IO));
+    rows(q + (tok * H_qk + hk) * D_K, D_K * (int)sizeof(IO));
+    rows(v + (tok * H_v + h) * D_V, D_V * (int)sizeof(IO));
+    if (CHANNEL_GATE) rows(g + (tok * H_v + h) * D_K, D_K * 4);
+  };
 
-  for (int t = 0; t < T; ++t) {
-    const int buf = t % 3, par = t & 1;
-    const bool more = t + 1 < T;
-    // prefetch token t+1's inputs into registers
-    float kn = 0.f, qn = 0.f, gn = 0.f, vn[CPL], bn = 0.f;
-    if (more) {
-      load_v(t + 1, vn, bn);
-      if (threadIdx.x < D_K) load_raw(t + 1, kn, qn, gn);
-    }
-
-    // 2. partial column sums over this warp's rows: r = S^T kr, p = S^T (a.q)
-    float rp[CPL], pp[CPL];
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) rp[c] = pp[c] = 0.f;
-#pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      const float ki = tv.kr[buf][warp * RPW + r], aqi = tv.aq[buf][warp * RPW + r];
-#pragma unroll
-      for (int c = 0; c < CPL; ++c) {
-        rp[c] = fmaf(ki, x[r][c], rp[c]);
-        pp[c] = fmaf(aqi, x[r][c], pp[c]);
-      }
-    }
-#pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      s_red[par][0][warp][lane * CPL + c] = rp[c];
-      s_red[par][1][warp][lane * CPL + c] = pp[c];
-    }
-    // token t+1's vectors go into the buffer token t-2 used (free by now)
-    if (more && threadIdx.x < D_K) stage((t + 1) % 3, kn, qn, gn, bn);
+  const int ocol = warp * CW + (lane % CW), opart = lane / CW;
+  for (int t0 = 0; t0 < T; t0 += TB) {
+    const int nt = (T - t0) < TB ? (T - t0) : TB;
+    if (!SINGLE) __syncthreads();  // the previous block's vectors are no longer read
+    if (warp < nt) stage(warp, t0 + warp);
+    if (!SINGLE && t0 + TB + warp < T) prefetch_token(t0 + TB + warp);
     __syncthreads();
 
-    float rf[CPL];
+    for (int tt = 0; tt < nt; ++tt) {
+      const int par = (t0 + tt) & 1;
+      // 2. partial column sums over this warp's rows: r = S^T kr, p = S^T (a.q)
+      float rp[CPL], pp[CPL];
 #pragma unroll
-    for (int c = 0; c < CPL; ++c) {
-      float acc = 0.f;
+      for (int c = 0; c < CPL; ++c) rp[c] = pp[c] = 0.f;
 #pragma unroll
-      for (int w = 0; w < kWarps; ++w) acc += s_red[par][0][w][lane * CPL + c];
-      rf[c] = acc;
-    }
-    if (more && threadIdx.x == 32) {  // token t+1's readout coefficients
-      float kq = 0.f, kaq = 0.f;
+      for (int r = 0; r < RPW; ++r) {
+        const float ki = bv.kr[tt][warp * RPW + r], aqi = bv.aq[tt][warp * RPW + r];
 #pragma unroll
-      for (int w = 0; w < D_K / 32; ++w) {
-        kq += s_dot[(t + 1) % 3][w][0];
-        kaq += s_dot[(t + 1) % 3][w][1];
+        for (int c = 0; c < CPL; ++c) {
+          rp[c] = fmaf(ki, x[r][c], rp[c]);
+          pp[c] = fmaf(aqi, x[r][c], pp[c]);
+        }
       }
-      tv.coef[(t + 1) % 3][0] = bn * (DECAY_FIRST ? kq : kaq);
-      tv.coef[(t + 1) % 3][1] = bn * kq;
-    }
+      vec<CPL>::sts(&s_red[par][0][warp][lane * CPL], rp);
+      vec<CPL>::sts(&s_red[par][1][warp][lane * CPL], pp);
+      __syncthreads();
 
-    // 3. S' = a . S - e r^T + beta k v^T (e folds the order), in registers
+      float rf[CPL], vv[CPL];
 #pragma unroll
-    for (int r = 0; r < RPW; ++r) {
-      const int i = warp * RPW + r;
-      const float a = tv.a[buf][i], e = tv.e[buf][i], bk = tv.bk[buf][i];
+      for (int c = 0; c < CPL; ++c) rf[c] = 0.f;
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) x[r][c] = fmaf(a, x[r][c], fmaf(-e, rf[c], bk * vv[c]));
-    }
-
-    // 4. o = p - c_r r + c_v v
-    if (warp == 0) {
-      const float cr = tv.coef[buf][0], cv = tv.coef[buf][1];
+      for (int w = 0; w < kWarps; ++w) {
+        float part[CPL];
+        vec<CPL>::lds(&s_red[par][0][w][lane * CPL], part);
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) {
-        float p = 0.f;
-#pragma unroll
-        for (int w = 0; w < kWarps; ++w) p += s_red[par][1][w][lane * CPL + c];
-        const float out = p - cr * rf[c] + cv * vv[c];
-        io<IO>::store(o + (token_base(t) * H_v + h) * D_V + lane * CPL + c, out);
+        for (int c = 0; c < CPL; ++c) rf[c] += part[c];
       }
-    }
-    if (more) {
+      vec<CPL>::lds(&bv.v[tt][lane * CPL], vv);
+
+      // 3. S' = a . S - e r^T + beta k v^T (e folds the order), in registers
 #pragma unroll
-      for (int c = 0; c < CPL; ++c) vv[c] = vn[c];
+      for (int r = 0; r < RPW; ++r) {
+        const int i = warp * RPW + r;
+        const float a = bv.a[tt][i], e = bv.e[tt][i], bk = bv.bk[tt][i];
+#pragma unroll
+        for (int c = 0; c < CPL; ++c) x[r][c] = fmaf(a, x[r][c], fmaf(-e, rf[c], bk * vv[c]));
+        if (SINGLE) vec<CPL>::st(S + i * D_V + lane * CPL, x[r]);
+      }
+
+      // 4. o = p - c_r r + c_v v, every warp a slice of the columns
+      float ps = 0.f, rs = 0.f;
+#pragma unroll
+      for (int w = 0; w < WPP; ++w) {
+        ps += s_red[par][1][opart * WPP + w][ocol];
+        rs += s_red[par][0][opart * WPP + w][ocol];
+      }
+#pragma unroll
+      for (int off = CW; off < 32; off <<= 1) {
+        ps += __shfl_xor_sync(0xffffffffu, ps, off);
+        rs += __shfl_xor_sync(0xffffffffu, rs, off);
+      }
+      if (opart == 0)
+        io<IO>::store(o + (token_base(t0 + tt) * H_v + h) * D_V + ocol,
+                      ps - bv.coef[tt][0] * rs + bv.coef[tt][1] * bv.v[tt][ocol]);
     }
   }
 
   // 5. the state goes back once, in place
+  if (!SINGLE) {
 #pragma unroll
-  for (int r = 0; r < RPW; ++r) vec<CPL>::st(S + (warp * RPW + r) * D_V + lane * CPL, x[r]);
+    for (int r = 0; r < RPW; ++r) vec<CPL>::st(S + (warp * RPW + r) * D_V + lane * CPL, x[r]);
+  }
 }
 
 template <int D_K, int D_V, typename IO>
@@ -258,12 +267,21 @@ cudaError_t launch_dv(const DecodeArgs &a, cudaStream_t s) {
 #define GDR_RECURRENT_ARGS                                                                  \
   (const IO *)a.q, (const IO *)a.k, (const IO *)a.v, a.g, a.beta, (IO *)a.o, a.state, a.slots, \
       a.num_slots, a.T, a.H_qk, a.H_v
-  if (!a.channel_gate)
-    recurrent_kernel<D_K, D_V, IO, false, false><<<grid, block, 0, s>>>(GDR_RECURRENT_ARGS);
-  else if (a.decay_first)
-    recurrent_kernel<D_K, D_V, IO, true, true><<<grid, block, 0, s>>>(GDR_RECURRENT_ARGS);
-  else
-    recurrent_kernel<D_K, D_V, IO, true, false><<<grid, block, 0, s>>>(GDR_RECURRENT_ARGS);
+  if (a.T == 1) {
+    if (!a.channel_gate)
+      recurrent_kernel<D_K, D_V, IO, false, false, true><<<grid, block, 0, s>>>(GDR_RECURRENT_ARGS);
+    else if (a.decay_first)
+      recurrent_kernel<D_K, D_V, IO, true, true, true><<<grid, block, 0, s>>>(GDR_RECURRENT_ARGS);
+    else
+      recurrent_kernel<D_K, D_V, IO, true, false, true><<<grid, block, 0, s>>>(GDR_RECURRENT_ARGS);
+  } else {
+    if (!a.channel_gate)
+      recurrent_kernel<D_K, D_V, IO, false, false, false><<<grid, block, 0, s>>>(GDR_RECURRENT_ARGS);
+    else if (a.decay_first)
+      recurrent_kernel<D_K, D_V, IO, true, true, false><<<grid, block, 0, s>>>(GDR_RECURRENT_ARGS);
+    else
+      recurrent_kernel<D_K, D_V, IO, true, false, false><<<grid, block, 0, s>>>(GDR_RECURRENT_ARGS);
+  }
 #undef GDR_RECURRENT_ARGS
   return cudaGetLastError();
 }
