@@ -187,7 +187,9 @@ constexpr uint32_t MISC_GSUM = 2560;   // f32[4][128] sum of g over each sub-chu
 constexpr uint32_t MISC_GLE = 4608;    // f32[128] e^{G_L}
 constexpr uint32_t MISC_BAR = 5120;    // 2 x u64
 constexpr uint32_t MISC_TSLOT = 5136;  // u32
-constexpr uint32_t PREP_SMEM = OFF_MISC + 6144 + 1024;
+constexpr uint32_t MISC_XP = 6144;     // f32[4][2][128] product of a over each half sub-chunk
+constexpr uint32_t MISC_XS = 10240;    // f32[4][2][128] sum of g over each half sub-chunk
+constexpr uint32_t PREP_SMEM = OFF_MISC + 14336 + 1024;
 constexpr uint32_t OFF_KAB = OFF_G, OFF_KBB = OFF_G + 16384;
 
 // X region, gram phase
@@ -207,9 +209,13 @@ constexpr uint32_t X_TINVF = 50176;   // 17 KB f32 [64][LDN]  (T^{-1}); both dea
 constexpr uint32_t X_W = 32768;       // after T2: K-major [c][t]
 constexpr uint32_t X_Y = 49152;       // after T2: K-major [n][t]
 constexpr uint32_t X_U = 65536;       // after T3: K-major [n][t]
-constexpr uint32_t X_QPI = 0;         // after T3: Q' image (16 KB), bulk-copied to the slot
-constexpr uint32_t X_PI = 81920;      // after T3: P image (32 KB); after T4: Qc image
-constexpr uint32_t X_OII = 0;         // after T4: O_intra image (16 KB)
+// slot images, staged in shared memory and bulk-copied to the workspace; the
+// copies' reads of these bytes only have to finish before the next item's
+// operand build
+constexpr uint32_t X_QPI = 0;         // after T4 issue: Q' image (16 KB)
+constexpr uint32_t X_PI = 81920;      // after T4 issue: P image (32 KB)
+constexpr uint32_t X_QCI = 16384;     // after T4: Qc image (32 KB)
+constexpr uint32_t X_OII = 49152;     // after T4: O_intra image (16 KB)
 
 // TMEM columns
 constexpr uint32_t TM_GRAM = 0, TM_P = 0, TM_W = 128, TM_QC = 128, TM_YB = 192, TM_OI = 256,
@@ -232,6 +238,56 @@ __device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
 }
 
 __device__ __forceinline__ void st16(unsigned char *p, uint4 v) { *reinterpret_cast<uint4 *>(p) = v; }
+
+
+// ---- warp-level tf32 MMA (m16n8k8) for the small block products of T^{-1} ----
+constexpr int LDT = 40;  // row stride (floats) of the fp32 scratch: conflict-free B fragments
+
+__device__ __forceinline__ uint32_t to_tf32(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return r;
+}
+
+// d (16x8 fp32, per-lane fragment) += A[0..16)[k] * B[k][n0 .. n0+8) over k in [k_lo, k_hi)
+// (multiples of 8).  A and B are row-major fp32 in shared memory with row
+// strides lda, ldb; A points at row 0 / column 0 of the tile, B at row 0 and
+// column n0 is given separately.  Fragments follow the m16n8k8 layout: lane =
+// 4 g + t holds A (g, t), (g+8, t), (g, t+4), (g+8, t+4), B (t, g), (t+4, g) and
+// D (g, 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1).
+__device__ __forceinline__ void warp_mma_tf32_range(float (&d)[4], const float *A, int lda,
+                                                    const float *B, int ldb, int n0, int k_lo,
+                                                    int k_hi, int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  for (int k0 = k_lo; k0 < k_hi; k0 += 8) {
+    const uint32_t a0 = to_tf32(A[g * lda + k0 + t]), a1 = to_tf32(A[(g + 8) * lda + k0 + t]);
+    const uint32_t a2 = to_tf32(A[g * lda + k0 + t + 4]), a3 = to_tf32(A[(g + 8) * lda + k0 + t + 4]);
+    const uint32_t b0 = to_tf32(B[(k0 + t) * ldb + n0 + g]), b1 = to_tf32(B[(k0 + t + 4) * ldb + n0 + g]);
+    asm volatile(
+        "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
+        "{%8, %9}, {%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+  }
+}
+
+// K-extent K from 0, B already offset to its column n0 (so n0 = 0 inside)
+template <int K>
+__device__ __forceinline__ void warp_mma_tf32(float (&d)[4], const float *A, int lda, const float *B,
+                                              int ldb, int lane) {
+  warp_mma_tf32_range(d, A, lda, B, ldb, 0, 0, K, lane);
+}
+
+// Writes a 16x8 fp32 fragment to row-major shared memory at P (row stride ld).
+__device__ __forceinline__ void store_frag(float *P, int ld, const float (&d)[4], int lane) {
+  const int g = lane >> 2, t = lane & 3;
+  *reinterpret_cast<float2 *>(P + g * ld + 2 * t) = make_float2(d[0], d[1]);
+  *reinterpret_cast<float2 *>(P + (g + 8) * ld + 2 * t) = make_float2(d[2], d[3]);
+}
+
+__device__ __forceinline__ void named_bar_sync(int id, int threads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
 
 template <bool CHANNEL, bool DECAY_FIRST>
 __global__ void __launch_bounds__(kPrepThreads, 1)
@@ -280,9 +336,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const uint32_t tm = *tslot;
 
   // ---- 1. TMA loads of an item's q, k, v (bf16, swizzled) and g (fp32) ----
-  auto issue_loads = [&](int w) {  // thread 0
+  // Items' chunk-table entries are read one item ahead of their use, so no
+  // thread waits on a global load between phases.
+  auto entry = [&](int w) { return w < total ? tab[w / H_v] : ChunkEntry{0, 0, 0, 0}; };
+  auto issue_loads = [&](int w, const ChunkEntry &e) {  // thread 0
     const int ck = w / H_v, hh = w - ck * H_v, hkk = hh / (H_v / H_qk);
-    const int ts = tab[ck].start;
+    const int ts = e.start;
+    (void)ck;
     fence_async_smem();
     mbar_arrive_expect_tx(bar_tma, 3 * 16384 + (CHANNEL ? 32768 : 0));
 #pragma unroll
@@ -293,9 +353,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     if (CHANNEL) tma_load_3d(sG, &tm_g, 0, hh, ts, bar_tma);
   };
-  auto prefetch_l2 = [&](int w) {  // thread 0: a later item's tiles into L2
+  auto prefetch_l2 = [&](int w, const ChunkEntry &e) {  // thread 0: a later item's tiles into L2
     const int ck = w / H_v, hh = w - ck * H_v, hkk = hh / (H_v / H_qk);
-    const int ts = tab[ck].start;
+    const int ts = e.start;
+    (void)ck;
 #pragma unroll
     for (int cb = 0; cb < 2; ++cb) {
       tma_prefetch_l2_3d(&tm_q, cb * 64, hkk, ts);
@@ -304,34 +365,46 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
     if (CHANNEL) tma_prefetch_l2_3d(&tm_g, 0, hh, ts);
   };
+  // beta (and the scalar gate) of an item, one token per thread tid < C
+  auto load_beta = [&](int w, const ChunkEntry &e, float &b, float &gs) {
+    const int hh = w % H_v;
+    b = (tid < e.len) ? __ldg(beta + (size_t)(e.start + tid) * H_v + hh) : 0.f;
+    gs = (!CHANNEL && tid < e.len) ? __ldg(g_scalar + (size_t)(e.start + tid) * H_v + hh) : 0.f;
+  };
+  float nbeta = 0.f, ngsc = 0.f;  // the coming item's, loaded one item ahead
+  ChunkEntry ce = entry(work), ce_next = entry(work + gridDim.x);
   if (tid == 0) {
-    issue_loads(work);
-    if (work + (int)gridDim.x < total) prefetch_l2(work + gridDim.x);
+    issue_loads(work, ce);
+    if (work + (int)gridDim.x < total) prefetch_l2(work + gridDim.x, ce_next);
   }
+  if (tid < C) load_beta(work, ce, nbeta, ngsc);
 
   for (int it = 0; work < total; ++it, work += gridDim.x) {
   const int chunk = work / H_v, h = work - chunk * H_v;
-  const ChunkEntry ce = tab[chunk];
-  const int L = ce.len, t0 = ce.start;
+  const int L = ce.len;
   unsigned char *slot = slots + ((size_t)chunk * H_v + h) * SLOT_BYTES;
   const int next = work + gridDim.x;
+  const ChunkEntry ce_next2 = entry(next + gridDim.x);  // used by the next item's prefetch
 
   if (tid < C) {
-    sBeta[tid] = (tid < L) ? __ldg(beta + (size_t)(t0 + tid) * H_v + h) : 0.f;
-    if (!CHANNEL) sGsc[tid] = (tid < L) ? __ldg(g_scalar + (size_t)(t0 + tid) * H_v + h) : 0.f;
+    sBeta[tid] = nbeta;
+    if (!CHANNEL) sGsc[tid] = ngsc;
   }
   mbar_wait(bar_tma, it & 1, hdr, KDA_DEVICE_TIMEOUT);
   __syncthreads();
 
   // ---- 2. per-token decays a = e^{g} (rows >= L: no decay), sub-chunk sums ----
-  // Thread (I, p, h) owns channels c = 2p, 2p+1 of tokens 8h .. 8h+7 of
-  // sub-chunk I; its neighbour lane (h ^ 1) owns the other half.  Every
+  // Thread (I, h, p) owns channels c = 2p, 2p+1 of tokens 8h .. 8h+7 of
+  // sub-chunk I; a warp spans 64 channels of the same rows, so its 4-byte
+  // stores below fill whole 128-byte rows (no bank conflicts).  The two
+  // halves of a sub-chunk exchange their partial products through shared
+  // memory.  Every
   // in-chunk factor is a product of these a's: with G the in-chunk cumulative
   // log-decay and E_I its value at the end of sub-chunk I,
   //   e^{G_t - E_{I-1}} = prefix product of a in sub-chunk I up to t   (<= 1)
   //   e^{E_I - G_t}     = suffix product after t                       (<= 1)
   // and factors across sub-chunks are products of whole-sub-chunk products.
-  const int bI = tid >> 7, c2 = ((tid >> 1) & 63) * 2, rh = tid & 1;
+  const int bI = tid >> 7, rh = (tid >> 6) & 1, c2 = (tid & 63) * 2;
   float a0[8], a1[8];
   float pre0, pre1, suf0, suf1;  // product of a before / after this thread's rows
   {
@@ -356,8 +429,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       p0 *= a0[r];
       p1 *= a1[r];
     }
-    const float op0 = __shfl_xor_sync(0xffffffffu, p0, 1), op1 = __shfl_xor_sync(0xffffffffu, p1, 1);
-    const float os0 = __shfl_xor_sync(0xffffffffu, s0, 1), os1 = __shfl_xor_sync(0xffffffffu, s1, 1);
+    float *xp = reinterpret_cast<float *>(sm + OFF_MISC + MISC_XP);
+    float *xs = reinterpret_cast<float *>(sm + OFF_MISC + MISC_XS);
+    *reinterpret_cast<float2 *>(xp + (2 * bI + rh) * DK + c2) = make_float2(p0, p1);
+    *reinterpret_cast<float2 *>(xs + (2 * bI + rh) * DK + c2) = make_float2(s0, s1);
+    __syncthreads();
+    const float2 op = *reinterpret_cast<const float2 *>(xp + (2 * bI + (rh ^ 1)) * DK + c2);
+    const float2 os = *reinterpret_cast<const float2 *>(xs + (2 * bI + (rh ^ 1)) * DK + c2);
+    const float op0 = op.x, op1 = op.y, os0 = os.x, os1 = os.y;
     pre0 = rh ? op0 : 1.f;
     pre1 = rh ? op1 : 1.f;
     suf0 = rh ? 1.f : op0;
@@ -369,6 +448,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       sGsum[bI * DK + c2 + 1] = s1 + os1;
     }
   }
+  // the previous item's image copies must have read the X region before it is rebuilt
+  if (tid == 0) bulk_wait_read0();
   __syncthreads();  // g is consumed: its region is reused below
 
   // ---- 3. one pass builds every operand of the chunk ----
@@ -533,86 +614,78 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
 
   // ---- 6. T^{-1}, T = I + N, N = tril_{-1}(A_e) diag(beta) (blocked, fp32) ----
+  // Unit lower triangular, so T^{-1} is built block by block:
+  //   diagonal 16x16 blocks by forward substitution (fp32, one thread per column);
+  //   T^{-1}[h][l] = -T^{-1}[h][h] N[h][l] T^{-1}[l][l] for the 16x16 blocks below
+  //   the diagonal pairs, then for the lower-left 32x32 block.  The block
+  //   products are warp-level tf32 MMAs with fp32 accumulation: too small for
+  //   the CTA-wide tensor-core path, and tf32 (10-bit mantissa) keeps them well
+  //   inside the bf16 rounding every T^{-1} entry gets afterwards.
   {
     const float *nae = reinterpret_cast<const float *>(sX + X_NAE);
     float *tinv = reinterpret_cast<float *>(sX + X_TINVF);
-    float *tmp = reinterpret_cast<float *>(sX + X_TINVB);  // 32 x 32 f32 scratch
-    // (a) the four 16x16 diagonal blocks, one warp each: column sweep
-    //     X = I;  for j: X[r][:] -= N[r][j] X[j][:]  (r > j); lane owns row
-    //     lane/2, columns 8*(lane&1) .. +8, row j is broadcast by shuffles.
-    if (warp < 4) {
-      const int B0 = 16 * warp, r = lane >> 1, c0 = 8 * (lane & 1);
-      float x[8];
+    float *tmp = reinterpret_cast<float *>(sX + X_TINVB);  // fp32 scratch, row stride LDT
+    // (a) column c of the inverse of diagonal block b: x_i = [i == c] - sum_{j<i} N_ij x_j
+    if (tid < 64) {
+      const int b = tid >> 4, c = tid & 15;
+      const float *nb = nae + 16 * b * LDN + 16 * b;
+      float x[16];
+      x[0] = (c == 0) ? 1.f : 0.f;
 #pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = (r == c0 + u) ? 1.f : 0.f;
-      float nrow[16];
+      for (int i = 1; i < 16; ++i) {
+        float row[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) nrow[j] = nae[(B0 + r) * LDN + B0 + j];
-#pragma unroll
-      for (int j = 0; j < 15; ++j) {
-        const float m = (r > j) ? nrow[j] : 0.f;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          const float xj = __shfl_sync(0xffffffffu, x[u], 2 * j + (lane & 1));
-          x[u] = fmaf(-m, xj, x[u]);
+        for (int q4 = 0; q4 < (i + 3) / 4; ++q4) {
+          const float4 r4 = *reinterpret_cast<const float4 *>(nb + i * LDN + 4 * q4);
+          row[4 * q4] = r4.x; row[4 * q4 + 1] = r4.y; row[4 * q4 + 2] = r4.z; row[4 * q4 + 3] = r4.w;
         }
+        float acc = (i == c) ? 1.f : 0.f;
+#pragma unroll
+        for (int j = 0; j < i - 1; ++j) acc = fmaf(-row[j], x[j], acc);
+        x[i] = fmaf(-row[i - 1], x[i - 1], acc);  // the newest term last: short chain
       }
 #pragma unroll
-      for (int u = 0; u < 8; ++u) tinv[(B0 + r) * LDN + B0 + c0 + u] = x[u];
-    }
-    // zero the strictly upper blocks
-    for (int e = tid; e < 64 * 64; e += kPrepThreads) {
-      const int rr = e >> 6, cc = e & 63;
-      if ((cc >> 4) > (rr >> 4)) tinv[rr * LDN + cc] = 0.f;
+      for (int i = 0; i < 16; ++i) tinv[(16 * b + i) * LDN + 16 * b + c] = x[i];
     }
     __syncthreads();
-    // (b) 32x32 level: T^{-1}[2p+1][2p] = -T^{-1}[2p+1][2p+1] N[2p+1][2p] T^{-1}[2p][2p]
-    {
-      const int pp = tid >> 8, r = (tid >> 4) & 15, cc = tid & 15;
-      const int R0 = 32 * pp + 16, C0 = 32 * pp;  // block row / column offsets
-      float acc = 0.f;
-#pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2)
-        acc = fmaf(nae[(R0 + r) * LDN + C0 + s2], tinv[(C0 + s2) * LDN + C0 + cc], acc);
-      tmp[(16 * pp + r) * 32 + cc] = acc;
-      __syncthreads();
-      acc = 0.f;
-#pragma unroll
-      for (int s2 = 0; s2 < 16; ++s2)
-        acc = fmaf(tinv[(R0 + r) * LDN + R0 + s2], tmp[(16 * pp + s2) * 32 + cc], acc);
-      tinv[(R0 + r) * LDN + C0 + cc] = -acc;
-      __syncthreads();
+    // (b) the two 16x16 blocks T^{-1}[16p+16][16p] (p = 0, 2): warp w < 4 owns
+    //     pair w >> 1 and 8 output columns (w & 1)
+    if (warp < 4) {
+      const int R0 = 32 * (warp >> 1) + 16, C0 = R0 - 16, n0 = 8 * (warp & 1);
+      float *tp = tmp + (warp >> 1) * 16 * LDT;
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      warp_mma_tf32<16>(d, nae + R0 * LDN + C0, LDN, tinv + C0 * LDN + C0 + n0, LDN, lane);
+      store_frag(tp + n0, LDT, d, lane);
+      named_bar_sync(1, 128);
+      float e[4] = {0.f, 0.f, 0.f, 0.f};
+      warp_mma_tf32<16>(e, tinv + R0 * LDN + R0, LDN, tp + n0, LDT, lane);
+      e[0] = -e[0]; e[1] = -e[1]; e[2] = -e[2]; e[3] = -e[3];
+      store_frag(tinv + R0 * LDN + C0 + n0, LDN, e, lane);
     }
-    // (c) 64x64 level: T^{-1}[lo][hi] = -T^{-1}[lo][lo] N[lo][hi] T^{-1}[hi][hi] (32x32 blocks)
-    {
-      const int r = tid >> 4, cq = (tid & 15) * 2;
-      float acc0 = 0.f, acc1 = 0.f;
-#pragma unroll 8
-      for (int s2 = 0; s2 < 32; ++s2) {
-        const float nv = nae[(32 + r) * LDN + s2];
-        const float2 tv = *reinterpret_cast<const float2 *>(tinv + s2 * LDN + cq);
-        acc0 = fmaf(nv, tv.x, acc0);
-        acc1 = fmaf(nv, tv.y, acc1);
-      }
-      *reinterpret_cast<float2 *>(tmp + r * 32 + cq) = make_float2(acc0, acc1);
-      __syncthreads();
-      acc0 = acc1 = 0.f;
-#pragma unroll 8
-      for (int s2 = 0; s2 < 32; ++s2) {
-        const float tv = tinv[(32 + r) * LDN + 32 + s2];
-        const float2 xv = *reinterpret_cast<const float2 *>(tmp + s2 * 32 + cq);
-        acc0 = fmaf(tv, xv.x, acc0);
-        acc1 = fmaf(tv, xv.y, acc1);
-      }
-      *reinterpret_cast<float2 *>(tinv + (32 + r) * LDN + cq) = make_float2(-acc0, -acc1);
-      __syncthreads();
+    __syncthreads();
+    // (c) the lower-left 32x32 block: warp w < 8 owns rows 16 (w >> 2) .. +16 and
+    //     columns 8 (w & 3) .. +8; zero blocks of the triangular factors are skipped
+    if (warp < 8) {
+      const int m0 = 16 * (warp >> 2), n0 = 8 * (warp & 3);
+      float d[4] = {0.f, 0.f, 0.f, 0.f};
+      // tmp = N[32..63][0..31] T^{-1}[0..31][0..31]: rows k < n0 of the right factor are 0
+      warp_mma_tf32_range(d, nae + (32 + m0) * LDN, LDN, tinv, LDN, n0, n0 & ~7, 32, lane);
+      store_frag(tmp + m0 * LDT + n0, LDT, d, lane);
+      named_bar_sync(1, 256);
+      float e[4] = {0.f, 0.f, 0.f, 0.f};
+      // T^{-1}[32..63][32..63] tmp: columns k >= m0 + 16 of the left factor are 0
+      warp_mma_tf32_range(e, tinv + (32 + m0) * LDN + 32, LDN, tmp, LDT, n0, 0, m0 + 16, lane);
+      e[0] = -e[0]; e[1] = -e[1]; e[2] = -e[2]; e[3] = -e[3];
+      store_frag(tinv + (32 + m0) * LDN + n0, LDN, e, lane);
     }
-    // bf16 copy, K-major [i][j]
+    __syncthreads();
+    // bf16 copy, K-major [i][j]; blocks above the diagonal are zero
     for (int item = tid; item < 64 * 8; item += kPrepThreads) {
       const int i = item >> 3, j = (item & 7) * 8;
       float x[8];
+      const bool upper = (j >> 4) > (i >> 4);
 #pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = tinv[i * LDN + j + u];
+      for (int u = 0; u < 8; ++u) x[u] = upper ? 0.f : tinv[i * LDN + j + u];
       st16(sX + X_TINVB + kmajor_off(i, j), pack8(x));
     }
   }
@@ -684,12 +757,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   tc_fence_after();
 
   {
-    float v[32];
-    // U (lanes n, cols t) -> K-major [n][t]
-    float u16[16], x16[16];
+    // U (lanes n, cols t) -> K-major [n][t], the left operand of the last products
+    float u16[16];
     tmem_ld16(taddr(tm, 32 * quad, TM_U + 16 * qtr), u16);
-    tmem_ld32(taddr(tm, 32 * quad, TM_P + 32 * qtr), v);
-    tmem_ld16(taddr(tm, 32 * quad, TM_X + 16 * qtr), x16);
     tmem_ld_wait();
 #pragma unroll
     for (int seg = 0; seg < 2; ++seg) {
@@ -698,6 +768,38 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       for (int u = 0; u < 8; ++u) x[u] = u16[8 * seg + u];
       st16(sX + X_U + kmajor_off(lane_row, 16 * qtr + 8 * seg), pack8(x));
     }
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  // ---- 9. O_intra^T -= U^T (B_e beta)^T;  Qc^T = V^T beta K_a - U^T beta K_b ----
+  if (tid == 0) {
+    const uint32_t usm = smem_u32(sX + X_U);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tm + TM_OI, desc_kmajor(usm, 16 * kk, 0), desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0),
+               idesc_bf16(128, 64, false, false, true), 1);
+    // Qc^T = V^T (beta K e^{G_L-G}) - U^T (beta K e^{G_L-Gp}): lanes j, columns i
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sV), 16 * kk, 8192),
+               desc_mnmajor(smem_u32(sm + OFF_KAB), 16 * kk, 8192), idesc_bf16(128, 128, true, true),
+               kk > 0);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tm + TM_QC, desc_kmajor(usm, 16 * kk, 0),
+               desc_mnmajor(smem_u32(sm + OFF_KBB), 16 * kk, 8192),
+               idesc_bf16(128, 128, false, true, true), 1);
+    mma_commit(bar_mma);
+  }
+  // P and Q' leave TMEM for the slot while the last products run (disjoint columns)
+  {
+    float v[32], x16[16];
+    tmem_ld32(taddr(tm, 32 * quad, TM_P + 32 * qtr), v);
+    tmem_ld16(taddr(tm, 32 * quad, TM_X + 16 * qtr), x16);
+    tmem_ld_wait();
     // P = Diag(e^{G_L}) - K_b^T beta W (lanes i, cols c) -> K-major A image [i][c]
     const int i = lane_row;
     const float gl = sGLe[i];
@@ -726,47 +828,24 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       st16(sX + X_QPI + sw128((uint32_t)(c * 128 + (16 * qtr + 8 * seg) * 2)), pack8(x));
     }
   }
+
   fence_async_smem();
-  tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  mbar_wait(bar_mma, 1, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
+  __syncthreads();  // the P / Q' images are written and every read of the q tile is done
+
   if (tid == 0) {  // P and Q' images -> workspace slot
     bulk_s2g(slot + SLOT_P, sX + X_PI, 32768);
     bulk_s2g(slot + SLOT_QP, sX + X_QPI, 16384);
     bulk_commit();
   }
-
-  // ---- 9. O_intra^T -= U^T (B_e beta)^T;  Qc^T = V^T beta K_a - U^T beta K_b ----
-  if (tid == 0) {
-    const uint32_t usm = smem_u32(sX + X_U);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_OI, desc_kmajor(usm, 16 * kk, 0), desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0),
-               idesc_bf16(128, 64, false, false, true), 1);
-    // Qc^T = V^T (beta K e^{G_L-G}) - U^T (beta K e^{G_L-Gp}): lanes j, columns i
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sV), 16 * kk, 8192),
-               desc_mnmajor(smem_u32(sm + OFF_KAB), 16 * kk, 8192), idesc_bf16(128, 128, true, true),
-               kk > 0);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_QC, desc_kmajor(usm, 16 * kk, 0),
-               desc_mnmajor(smem_u32(sm + OFF_KBB), 16 * kk, 8192),
-               idesc_bf16(128, 128, false, true, true), 1);
-    mma_commit(bar_mma);
-  }
-  __syncwarp();
-  mbar_wait(bar_mma, 1, hdr, KDA_DEVICE_TIMEOUT);
-  tc_fence_after();
-
   // the input tiles are consumed: start the next item's loads now
   if (tid == 0 && next < total) {
-    issue_loads(next);
-    if (next + (int)gridDim.x < total) prefetch_l2(next + gridDim.x);
+    issue_loads(next, ce_next);
+    if (next + (int)gridDim.x < total) prefetch_l2(next + gridDim.x, ce_next2);
   }
-  if (tid == 0) bulk_wait_read0();  // the P / Q' images may now be overwritten
-  __syncthreads();
+  if (tid < C && next < total) load_beta(next, ce_next, nbeta, ngsc);
   {
     float v[32];
     // O_intra^T (lanes j, cols t) -> image row-major [j][t]
@@ -788,21 +867,20 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       float x[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) x[u] = v[8 * seg + u];
-      st16(sX + X_PI + rowimg_off(j, DK * 2, 4 * qtr + seg), pack8(x));
+      st16(sX + X_QCI + rowimg_off(j, DK * 2, 4 * qtr + seg), pack8(x));
     }
   }
   fence_async_smem();
   tc_fence_before();
   __syncthreads();
-  if (tid == 0) {
-    bulk_s2g(slot + SLOT_QC, sX + X_PI, 32768);
+  tc_fence_after();
+  if (tid == 0) {  // Qc and O_intra images -> workspace slot
+    bulk_s2g(slot + SLOT_QC, sX + X_QCI, 32768);
     bulk_s2g(slot + SLOT_OI, sX + X_OII, 16384);
     bulk_commit();
-    bulk_wait_read0();  // the next item rebuilds over these images
   }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
+  ce = ce_next;
+  ce_next = ce_next2;
   }  // work items
 
   if (tid == 0) bulk_wait0();
