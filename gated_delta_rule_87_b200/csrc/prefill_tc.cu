@@ -70,33 +70,36 @@ struct ChunkEntry {
 constexpr size_t kHeaderBytes = 256;  // [0] status word, [1] number of chunks
 constexpr uint32_t SLOT_P = 0;        // 32 KB  P, K-major A image [i][c]
 constexpr uint32_t SLOT_QP = 32768;   // 16 KB  Q', MN-major A image [c][t]
-constexpr uint32_t SLOT_QC = 49152;   // 32 KB  Qc^T, bf16 row-major [j][i] (rowimg_off)
-constexpr uint32_t SLOT_OI = 81920;   // 16 KB  O_intra^T, bf16 row-major [j][t] (rowimg_off)
+constexpr uint32_t SLOT_QC = 49152;   // 32 KB  Qc, four 32-column slices [s][i][32 j] (slice_off)
+constexpr uint32_t SLOT_OI = 81920;   // 16 KB  O_intra, four 32-column slices [s][t][32 j] (slice_off)
 constexpr uint32_t SLOT_BYTES = 98304;
 
 size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
 
 struct WsLayout {
-  size_t seq_off, tab, slots, total;
+  size_t seq_off, order, tab, slots, total;
 };
 WsLayout ws_layout(int64_t T_total, int num_seqs) {
   WsLayout L;
   const int64_t max_chunks = T_total / C + num_seqs;
   L.seq_off = kHeaderBytes;
-  L.tab = align_up(L.seq_off + sizeof(int32_t) * ((size_t)num_seqs + 1), 256);
+  L.order = align_up(L.seq_off + sizeof(int32_t) * ((size_t)num_seqs + 1), 256);
+  L.tab = align_up(L.order + sizeof(int32_t) * (size_t)num_seqs, 256);
   L.slots = align_up(L.tab + sizeof(ChunkEntry) * (size_t)max_chunks, 1024);
   L.total = L.slots;  // + slots, added by the caller (depends on H_v)
   return L;
 }
 
 // ---------------------------------------------------------------------------
-// planning: chunk table and per-sequence chunk offsets (also validates
-// cu_seqlens)
+// planning: chunk table, per-sequence chunk offsets and the order in which
+// the scan takes the sequences (also validates cu_seqlens)
 // ---------------------------------------------------------------------------
+constexpr int kSortMax = 512;  // packed batches up to this size are scanned longest first
 __global__ void __launch_bounds__(1024, 1)
 plan_kernel(const int32_t *__restrict__ cu, int num_seqs, int T, int T_total, int32_t *hdr,
-            int32_t *seq_off, ChunkEntry *tab) {
+            int32_t *seq_off, int32_t *order, ChunkEntry *tab) {
   __shared__ int32_t warp_tot[32];
+  __shared__ int32_t s_len[kSortMax];
   __shared__ int32_t s_running;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   bool bad = false;
@@ -166,6 +169,22 @@ plan_kernel(const int32_t *__restrict__ cu, int num_seqs, int T, int T_total, in
     seq_off[num_seqs] = s_running;
     hdr[1] = s_running;
   }
+  // scan order: decreasing length (ties by index), so the longest chains start first
+  if (cu && num_seqs <= kSortMax) {
+    for (int i = tid; i < num_seqs; i += blockDim.x) s_len[i] = cu[i + 1] - cu[i];
+    __syncthreads();
+    for (int i = tid; i < num_seqs; i += blockDim.x) {
+      const int li = s_len[i];
+      int r = 0;
+      for (int m = 0; m < num_seqs; ++m) {
+        const int lm = s_len[m];
+        r += (lm > li) || (lm == li && m < i);
+      }
+      order[r] = i;
+    }
+  } else {
+    for (int i = tid; i < num_seqs; i += blockDim.x) order[i] = i;
+  }
 }
 
 // ---------------------------------------------------------------------------
@@ -217,20 +236,23 @@ constexpr uint32_t X_PI = 81920;      // after T4 issue: P image (32 KB)
 constexpr uint32_t X_QCI = 16384;     // after T4: Qc image (32 KB)
 constexpr uint32_t X_OII = 49152;     // after T4: O_intra image (16 KB)
 
-// TMEM columns
-constexpr uint32_t TM_GRAM = 0, TM_P = 0, TM_W = 128, TM_QC = 128, TM_YB = 192, TM_OI = 256,
-                   TM_U = 320, TM_X = 384;
+// TMEM columns (W, Y die at their readback, U at its readback)
+constexpr uint32_t TM_GRAM = 0, TM_P = 0, TM_OI = 128, TM_W = 256, TM_Y = 320, TM_U = 256,
+                   TM_QC = 256, TM_X = 384;
 
 __device__ __forceinline__ float ld_bf16(const unsigned char *base, uint32_t off) {
   return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(base + off));
 }
 
-// Row-major bf16 images read one row per thread (Qc^T, O_intra^T): the 16-byte
-// chunks of row j are XOR-swizzled by j mod 8 so that 32 threads reading 32
-// rows hit all banks.  Byte offset of chunk `ch` (8 elements) of row j:
-__device__ __forceinline__ uint32_t rowimg_off(int j, int row_bytes, int ch) {
-  return (uint32_t)(j * row_bytes + (((ch & ~7) | ((ch ^ j) & 7)) * 16));
+// Column-slice images read one row per thread (Qc, O_intra): 32 value columns
+// of bf16 per row (64 bytes), the 16-byte chunks swizzled as in the SW64
+// operand layout so that the 8 threads of a shared-memory phase hit distinct
+// banks.  Byte offset of chunk `ch` (columns 8 ch .. 8 ch + 7) of row r:
+__device__ __forceinline__ uint32_t slice_off(int r, int ch) {
+  return sw64((uint32_t)(r * 64 + ch * 16));
 }
+constexpr uint32_t QC_SLICE_BYTES = 128 * 64;  // d_k rows
+constexpr uint32_t OI_SLICE_BYTES = 64 * 64;   // C rows
 
 __device__ __forceinline__ uint4 pack8(const float (&x)[8]) {
   return make_uint4(pack_bf16x2(x[0], x[1]), pack_bf16x2(x[2], x[3]), pack_bf16x2(x[4], x[5]),
@@ -694,7 +716,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
   tc_fence_after();
 
-  // ---- 7. W^T = (K e^{Gp})^T T^{-T};  [Y^T | (B_w beta V)^T] = V^T [(A_w beta)^T | (B_w beta)^T] ----
+  // ---- 7. W^T = (K e^{Gp})^T T^{-T};  Y^T = V^T (A_w beta)^T ----
   if (tid == 0) {
     const uint32_t tinvb = smem_u32(sX + X_TINVB);
 #pragma unroll
@@ -703,8 +725,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
                desc_kmajor(tinvb, 16 * kk, 0), idesc_bf16(128, 64, true, false), kk > 0);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_YB, desc_mnmajor(smem_u32(sV), 16 * kk, 8192),
-               desc_kmajor(smem_u32(sX + X_AWBW), 16 * kk, 0), idesc_bf16(128, 128, true, false),
+      mma_bf16(tm + TM_Y, desc_mnmajor(smem_u32(sV), 16 * kk, 8192),
+               desc_kmajor(smem_u32(sX + X_AWBW), 16 * kk, 0), idesc_bf16(128, 64, true, false),
                kk > 0);
     mma_commit(bar_mma);
   }
@@ -716,7 +738,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   {
     float v[16], v2[16];
     tmem_ld16(taddr(tm, 32 * quad, TM_W + 16 * qtr), v);
-    tmem_ld16(taddr(tm, 32 * quad, TM_YB + 16 * qtr), v2);
+    tmem_ld16(taddr(tm, 32 * quad, TM_Y + 16 * qtr), v2);
     tmem_ld_wait();
 #pragma unroll
     for (int seg = 0; seg < 2; ++seg) {
@@ -735,9 +757,16 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
   tc_fence_after();
 
-  // ---- 8. U^T = Y^T T^{-T};  K_b^T beta W (for P);  X = W^T (B_e beta)^T (for Q') ----
+  // ---- 8. U^T = Y^T T^{-T};  K_b^T beta W (for P);  X = W^T (B_e beta)^T (for Q');
+  //         O_intra = tril(B_w) beta V (rows t < 64 of an M = 128 product whose
+  //         upper 64 rows read the bytes after the operand and are discarded) ----
   if (tid == 0) {
     const uint32_t tinvb = smem_u32(sX + X_TINVB), wsm = smem_u32(sX + X_W);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tm + TM_OI, desc_kmajor(smem_u32(sX + X_AWBW + 64 * 128), 16 * kk, 0),
+               desc_mnmajor(smem_u32(sV), 16 * kk, 8192), idesc_bf16(128, 128, false, true),
+               kk > 0);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_U, desc_kmajor(smem_u32(sX + X_Y), 16 * kk, 0), desc_kmajor(tinvb, 16 * kk, 0),
@@ -774,24 +803,23 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
   tc_fence_after();
 
-  // ---- 9. O_intra^T -= U^T (B_e beta)^T;  Qc^T = V^T beta K_a - U^T beta K_b ----
+  // ---- 9. O_intra -= tril(B_e) beta U (M = 128 as in step 8);
+  //         Qc = (beta K e^{G_L-G})^T V - (beta K e^{G_L-Gp})^T U: lanes i, columns j ----
   if (tid == 0) {
     const uint32_t usm = smem_u32(sX + X_U);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_OI, desc_kmajor(usm, 16 * kk, 0), desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0),
-               idesc_bf16(128, 64, false, false, true), 1);
-    // Qc^T = V^T (beta K e^{G_L-G}) - U^T (beta K e^{G_L-Gp}): lanes j, columns i
+      mma_bf16(tm + TM_OI, desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0), desc_kmajor(usm, 16 * kk, 0),
+               idesc_bf16(128, 128, false, false, true), 1);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sV), 16 * kk, 8192),
-               desc_mnmajor(smem_u32(sm + OFF_KAB), 16 * kk, 8192), idesc_bf16(128, 128, true, true),
+      mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sm + OFF_KAB), 16 * kk, 8192),
+               desc_mnmajor(smem_u32(sV), 16 * kk, 8192), idesc_bf16(128, 128, true, true),
                kk > 0);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_QC, desc_kmajor(usm, 16 * kk, 0),
-               desc_mnmajor(smem_u32(sm + OFF_KBB), 16 * kk, 8192),
-               idesc_bf16(128, 128, false, true, true), 1);
+      mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sm + OFF_KBB), 16 * kk, 8192),
+               desc_kmajor(usm, 16 * kk, 0), idesc_bf16(128, 128, true, false, true), 1);
     mma_commit(bar_mma);
   }
   // P and Q' leave TMEM for the slot while the last products run (disjoint columns)
@@ -847,27 +875,28 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   if (tid < C && next < total) load_beta(next, ce_next, nbeta, ngsc);
   {
+    // warp (quad, qtr) holds rows 32 quad + lane, value columns 32 qtr .. +31,
+    // i.e. one row of column slice qtr
     float v[32];
-    // O_intra^T (lanes j, cols t) -> image row-major [j][t]
-    const int j = lane_row;
-    float o16[16];
-    tmem_ld16(taddr(tm, 32 * quad, TM_OI + 16 * qtr), o16);
     tmem_ld32(taddr(tm, 32 * quad, TM_QC + 32 * qtr), v);
     tmem_ld_wait();
 #pragma unroll
-    for (int seg = 0; seg < 2; ++seg) {
-      float x[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = o16[8 * seg + u];
-      st16(sX + X_OII + rowimg_off(j, C * 2, 2 * qtr + seg), pack8(x));
-    }
-    // Qc^T (lanes j, cols i) -> image row-major [j][i]
-#pragma unroll
-    for (int seg = 0; seg < 4; ++seg) {
+    for (int seg = 0; seg < 4; ++seg) {  // Qc rows i
       float x[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) x[u] = v[8 * seg + u];
-      st16(sX + X_QCI + rowimg_off(j, DK * 2, 4 * qtr + seg), pack8(x));
+      st16(sX + X_QCI + qtr * QC_SLICE_BYTES + slice_off(lane_row, seg), pack8(x));
+    }
+    if (quad < 2) {  // O_intra rows t < 64 (lanes 64..127 hold the discarded rows)
+      tmem_ld32(taddr(tm, 32 * quad, TM_OI + 32 * qtr), v);
+      tmem_ld_wait();
+#pragma unroll
+      for (int seg = 0; seg < 4; ++seg) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = v[8 * seg + u];
+        st16(sX + X_OII + qtr * OI_SLICE_BYTES + slice_off(lane_row, seg), pack8(x));
+      }
     }
   }
   fence_async_smem();
@@ -892,238 +921,291 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 // ---------------------------------------------------------------------------
 // scan kernel
 // ---------------------------------------------------------------------------
-constexpr int NSTAGE = 2;
-constexpr uint32_t ST_P = 0, ST_QP = 32768, ST_QC = 49152, ST_OI = 81920, ST_BYTES = 98304;
-constexpr uint32_t SC_OT = NSTAGE * ST_BYTES;  // 16 KB output tile [t][j] bf16
-constexpr uint32_t SC_MISC = SC_OT + 16384;
-constexpr uint32_t SCAN_SMEM = SC_MISC + 256 + 1024;
-constexpr uint32_t STAGE_TX = SLOT_BYTES;
-// TMEM columns: S^T operand (bf16 pairs) x3, D_s = (P S)^T, D_o = (Q' S)^T x2
-constexpr uint32_t TA0 = 0, TD_S = 192, TD_O = 320;
-// warp roles
-constexpr int kChainWarps = 8;   // warps 0-7: state column j = lane quadrant, half of the rows
-constexpr int kOutWarps = 4;     // warps 8-11: outputs
-constexpr int kMmaWarp = 12;
-constexpr int kLoadWarp = 13;
-constexpr int kScanThreads = 32 * 14;
-constexpr int kOutBarrier = 1;   // named barrier among the output warps
+// The columns of the state never interact (every chunk map multiplies S from
+// the left), so a (sequence, v-head) chain is split into 128 / NS column
+// slices, one CTA each.  Per chunk u a CTA computes, for its NS columns,
+//     S_{u+1} = P_u S_u + Qc_u        o_u = Q'_u S_u + O_intra_u
+// with S_u in bf16 as the MN-major B operand in shared memory, P_u (K-major)
+// and Q'_u (MN-major, M padded to 128: rows t >= 64 read the next bytes of the
+// stage and land in TMEM lanes nobody reads) as A operands, fp32 accumulators
+// in TMEM and the fp32 state in registers of the chain warps.  Roles,
+// connected by mbarriers:
+//   chain warps 0-3 : S_{u+1} = (P S)_u + Qc_u, row i = TMEM lane i
+//   output warps 4-5: o_u = (Q' S)_u + O_intra_u, row t = TMEM lane t
+//   MMA warp 6      : the two products of each chunk
+//   load warp 7     : chunk slots into kStages stages (bulk copies)
+template <int NS>
+struct ScanCfg {
+  static constexpr int kSlices = NS / 32;   // 32-column image slices per CTA
+  static constexpr int kStages = NS == 32 ? 3 : 2;
+  static constexpr uint32_t QC_BYTES = QC_SLICE_BYTES * kSlices;
+  static constexpr uint32_t OI_BYTES = OI_SLICE_BYTES * kSlices;
+  static constexpr uint32_t ST_P = 0, ST_QP = 32768, ST_QC = 49152, ST_OI = ST_QC + QC_BYTES;
+  static constexpr uint32_t ST_BYTES = ST_OI + OI_BYTES;  // 60 KB / 72 KB
+  static constexpr uint32_t SB_BYTES = 128 * NS * 2;     // bf16 state operand [c][NS]
+  static constexpr uint32_t OFF_SB = kStages * ST_BYTES;  // two state operand buffers
+  static constexpr uint32_t OFF_MISC = OFF_SB + 2 * SB_BYTES;
+  static constexpr uint32_t SMEM = OFF_MISC + 256 + 1024;
+  static constexpr uint32_t TD_S = 0, TD_O = NS;          // TMEM columns: (P S), (Q' S) x 2
+  static constexpr uint32_t TMEM_COLS = NS == 32 ? 128 : 256;
+};
+constexpr int kScanThreads = 256;
+constexpr int kScanMmaWarp = 6, kScanLoadWarp = 7;
+constexpr uint32_t kScanEmptyCount = 128 + 64 + 1;  // chain + output threads + MMA commit
 
-// The scan walks one sequence's chunks for one v-head, computing the
-// transposed state S^T (lanes = value column j, d_k along TMEM columns):
-//     (S_{u+1})^T = S_u^T P_u^T + Qc_u^T ,      o_u^T = S_u^T Q'_u^T + O_intra_u^T
-// S_u^T lives in TMEM as the bf16 A operand, so the serial chain is
-//   tcgen05.ld (P S)^T -> + Qc^T -> tcgen05.st bf16 -> 8 MMAs (128x128x16)
-// and never touches shared memory.  Roles, connected by mbarriers:
-//   chain warps  : S^T update, rows [64*half, 64*half + 64) of lane j
-//   MMA warp     : P_u products, then the previous chunk's Q' product
-//   output warps : o_u = (D_o)^T + O_intra -> shared tile -> global
-//   load warp    : chunk inputs into NSTAGE stages (bulk copies)
+// byte offset of the 16-byte chunk `ch` of state-operand row c (MN-major, NS columns)
+template <int NS>
+__device__ __forceinline__ uint32_t sop_off(int c, int ch) {
+  return NS == 32 ? sw64((uint32_t)(c * 64 + ch * 16)) : sw128((uint32_t)(c * 128 + ch * 16));
+}
+template <int NS>
+__device__ __forceinline__ uint64_t sop_desc(uint32_t base, int kk) {
+  return NS == 32 ? desc_mnmajor32(base, 16 * kk) : desc_mnmajor(base, 16 * kk, 16384);
+}
+
+template <int NS>
 __global__ void __launch_bounds__(kScanThreads, 1)
 chunk_scan_kernel(const int32_t *hdr, const int32_t *__restrict__ seq_off,
-                  const ChunkEntry *__restrict__ tab, const unsigned char *__restrict__ slots,
-                  __nv_bfloat16 *__restrict__ o, const float *s0, float *sT,
-                  const int32_t *__restrict__ state_slots, int64_t num_slots, int H_v,
-                  int32_t *err) {
+                  const int32_t *__restrict__ order, const ChunkEntry *__restrict__ tab,
+                  const unsigned char *__restrict__ slots, __nv_bfloat16 *__restrict__ o,
+                  const float *s0, float *sT, const int32_t *__restrict__ state_slots,
+                  int64_t num_slots, int H_v, int32_t *err) {
+  using Cfg = ScanCfg<NS>;
+  constexpr int NSL = 128 / NS;  // CTAs per (sequence, v-head)
+  constexpr int S = Cfg::kStages;
   extern __shared__ unsigned char smem_raw[];
-  // 1024-byte aligned base, derived by pointer arithmetic on the shared array so
-  // that the compiler keeps shared-memory addressing for every access
   unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  uint64_t *full = reinterpret_cast<uint64_t *>(sm + SC_MISC);  // [NSTAGE]
-  uint64_t *empty = full + NSTAGE;                              // [NSTAGE], chain + out arrivals
-  uint64_t *op_ready = empty + NSTAGE;                          // [3], chain arrivals
-  uint64_t *o_free = op_ready + 3;                              // [2], out arrivals
-  uint64_t *bar_s = o_free + 2;                                 // commit
-  uint64_t *bar_o = bar_s + 1;                                  // [2], commit
-  uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + SC_MISC + 192);
+  uint64_t *full = reinterpret_cast<uint64_t *>(sm + Cfg::OFF_MISC);  // [S] loads landed
+  uint64_t *empty = full + S;         // [S] stage consumed (chain, output, MMA commit)
+  uint64_t *sb_ready = empty + S;     // [2] state operand written (chain)
+  uint64_t *ds_full = sb_ready + 2;   // (P S) done (commit)
+  uint64_t *do_full = ds_full + 1;    // [2] (Q' S) done (commit)
+  uint64_t *do_free = do_full + 2;    // [2] (Q' S) read (output)
+  uint64_t *drain = do_free + 2;      // final commit of the MMA warp
+  uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + Cfg::OFF_MISC + 192);
 
   if (hdr[0] != KDA_DEVICE_OK) return;
-  const int n = blockIdx.x, h = blockIdx.y;
+  const int cid = blockIdx.x;
+  const int sl = cid % NSL, h = (cid / NSL) % H_v;
+  const int n = order[cid / (NSL * H_v)];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c_begin = seq_off[n], c_end = seq_off[n + 1];
-  const int nch = c_end - c_begin;
+  const int c_begin = seq_off[n], nch = seq_off[n + 1] - c_begin;
 
   if (warp == 0) {
-    tmem_alloc(tslot, 512);
+    tmem_alloc(tslot, Cfg::TMEM_COLS);
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int st = 0; st < NSTAGE; ++st) {
+    for (int st = 0; st < S; ++st) {
       mbar_init(&full[st], 1);
-      mbar_init(&empty[st], 32 * (kChainWarps + kOutWarps));
+      mbar_init(&empty[st], kScanEmptyCount);
     }
-    for (int b = 0; b < 3; ++b) mbar_init(&op_ready[b], 32 * kChainWarps);
     for (int b = 0; b < 2; ++b) {
-      mbar_init(&o_free[b], 32 * kOutWarps);
-      mbar_init(&bar_o[b], 1);
+      mbar_init(&sb_ready[b], 128);
+      mbar_init(&do_full[b], 1);
+      mbar_init(&do_free[b], 64);
     }
-    mbar_init(bar_s, 1);
+    mbar_init(ds_full, 1);
+    mbar_init(drain, 1);
     mbar_fence_init();
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *tslot;
-  // the state's pool slot; a negative slot starts from zeros and keeps no final state
+  // the state's pool slot; a slot outside the pool starts from zeros and keeps no final state
   const int64_t sslot = state_slots ? (int64_t)state_slots[n] : (int64_t)n;
   if (sslot < 0 || sslot >= num_slots) {
     s0 = nullptr;
     sT = nullptr;
   }
-  const size_t state_base = ((size_t)sslot * H_v + h) * DK * DK;
+  const size_t state_base = ((size_t)sslot * H_v + h) * DK * DK + (size_t)sl * NS;
+  auto slot_of = [&](int u) {
+    return slots + ((size_t)(c_begin + u) * H_v + h) * SLOT_BYTES;
+  };
 
-  if (warp == kLoadWarp) {
+  if (warp == kScanLoadWarp) {
     // ---------------- loads ----------------
     if (lane == 0) {
       constexpr int kAhead = 4;  // chunks prefetched into L2 ahead of their stage load
-      for (int u = 0; u < kAhead && u < nch; ++u)
-        bulk_prefetch_l2(slots + ((size_t)(c_begin + u) * H_v + h) * SLOT_BYTES, SLOT_BYTES);
+      auto prefetch = [&](int u) {
+        const unsigned char *src = slot_of(u);
+        bulk_prefetch_l2(src + SLOT_P, 49152);  // P and Q'
+        bulk_prefetch_l2(src + SLOT_QC + sl * Cfg::QC_BYTES, Cfg::QC_BYTES);
+        bulk_prefetch_l2(src + SLOT_OI + sl * Cfg::OI_BYTES, Cfg::OI_BYTES);
+      };
+      for (int u = 0; u < kAhead && u < nch; ++u) prefetch(u);
+      int issued = 0;
       for (int u = 0; u < nch; ++u) {
-        const int st = u % NSTAGE;
-        if (u + kAhead < nch)
-          bulk_prefetch_l2(slots + ((size_t)(c_begin + u + kAhead) * H_v + h) * SLOT_BYTES,
-                           SLOT_BYTES);
-        if (u >= NSTAGE) mbar_wait(&empty[st], ((u - NSTAGE) / NSTAGE) & 1, err, KDA_DEVICE_TIMEOUT);
-        mbar_arrive_expect_tx(&full[st], STAGE_TX);
-        bulk_g2s(sm + st * ST_BYTES, slots + ((size_t)(c_begin + u) * H_v + h) * SLOT_BYTES,
-                 SLOT_BYTES, &full[st]);
+        const int st = u % S;
+        if (u + kAhead < nch) prefetch(u + kAhead);
+        if (u >= S && !mbar_wait(&empty[st], ((u / S) - 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
+        unsigned char *dst = sm + st * Cfg::ST_BYTES;
+        const unsigned char *src = slot_of(u);
+        mbar_arrive_expect_tx(&full[st], Cfg::ST_BYTES);
+        bulk_g2s(dst + Cfg::ST_P, src + SLOT_P, 49152, &full[st]);
+        bulk_g2s(dst + Cfg::ST_QC, src + SLOT_QC + sl * Cfg::QC_BYTES, Cfg::QC_BYTES, &full[st]);
+        bulk_g2s(dst + Cfg::ST_OI, src + SLOT_OI + sl * Cfg::OI_BYTES, Cfg::OI_BYTES, &full[st]);
+        issued = u + 1;
       }
+      // no copy may still be writing this CTA's shared memory when it exits
+      for (int u = (issued > S ? issued - S : 0); u < issued; ++u)
+        mbar_wait(&full[u % S], (u / S) & 1, err, KDA_DEVICE_TIMEOUT);
     }
-  } else if (warp == kMmaWarp) {
+  } else if (warp == kScanMmaWarp) {
     // ---------------- tensor-core issue ----------------
     if (lane == 0) {
-      auto q_product = [&](int u) {  // o_u^T = S_u^T Q'_u^T  (M = 128 j, N = 64 t)
-        const uint32_t qa = smem_u32(sm + (u % NSTAGE) * ST_BYTES + ST_QP);
-        if (u >= 2) mbar_wait(&o_free[u & 1], ((u - 2) >> 1) & 1, err, KDA_DEVICE_TIMEOUT);
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tm + TD_O + 64 * (u & 1), tm + TA0 + 64 * (u % 3) + 8 * kk,
-                      desc_mnmajor(qa, 16 * kk, 0), idesc_bf16(128, 64, false, true), kk > 0);
-        mma_commit(&bar_o[u & 1]);
-      };
+      constexpr uint32_t idS = idesc_bf16(128, NS, false, true);  // P K-major, S MN-major
+      constexpr uint32_t idO = idesc_bf16(128, NS, true, true);   // Q' MN-major, S MN-major
       for (int u = 0; u < nch; ++u) {
-        const int st = u % NSTAGE;
-        mbar_wait(&op_ready[u % 3], (u / 3) & 1, err, KDA_DEVICE_TIMEOUT);
-        mbar_wait(&full[st], (u / NSTAGE) & 1, err, KDA_DEVICE_TIMEOUT);
+        const int st = u % S, b = u & 1;
+        if (!mbar_wait(&sb_ready[b], (u >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
+        if (!mbar_wait(&full[st], (u / S) & 1, err, KDA_DEVICE_TIMEOUT)) break;
         tc_fence_after();
-        const uint32_t pa = smem_u32(sm + st * ST_BYTES + ST_P);
-        // (P S)^T = S^T P^T  (M = 128 j, N = 128 i, K = 128 c); B = P rows, K-major
+        const uint32_t stage = smem_u32(sm + st * Cfg::ST_BYTES);
+        const uint32_t sb = smem_u32(sm + Cfg::OFF_SB + b * Cfg::SB_BYTES);
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          mma_bf16_ts(tm + TD_S, tm + TA0 + 64 * (u % 3) + 8 * kk, desc_kmajor(pa, 16 * kk, 16384),
-                      idesc_bf16(128, 128, false, false), kk > 0);
-        mma_commit(bar_s);
-        q_product(u);  // overlaps the chain's state update
+          mma_bf16(tm + Cfg::TD_S, desc_kmajor(stage + Cfg::ST_P, 16 * kk, 16384),
+                   sop_desc<NS>(sb, kk), idS, kk > 0);
+        mma_commit(ds_full);
+        if (u >= 2 && !mbar_wait(&do_free[b], ((u - 2) >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tm + Cfg::TD_O + NS * b, desc_mnmajor(stage + Cfg::ST_QP, 16 * kk, 16384),
+                   sop_desc<NS>(sb, kk), idO, kk > 0);
+        mma_commit(&do_full[b]);
+        mma_commit(&empty[st]);
       }
+      // every issued product has finished before TMEM is released
+      mma_commit(drain);
+      mbar_wait(drain, 0, err, KDA_DEVICE_TIMEOUT);
     }
-  } else if (warp < kChainWarps) {
-    // ---------------- the state chain: column j, rows [64*hh, 64*hh + 64) ----------------
-    const int q4 = warp & 3, hh = warp >> 2;
-    const int j = 32 * q4 + lane;
-    float S[64];
+  } else if (warp < 4) {
+    // ---------------- the state chain: row i, NS columns ----------------
+    const int i = 32 * warp + lane;
+    float Sr[NS];
+    if (s0) {
 #pragma unroll
-    for (int r = 0; r < 64; ++r)
-      S[r] = s0 ? s0[state_base + (size_t)(64 * hh + r) * DK + j] : 0.f;
-    auto write_operand = [&](int buf) {  // S^T rows -> bf16 pairs in TMEM
-      uint32_t pk[32];
+      for (int j = 0; j < NS; j += 4) {
+        const float4 x = *reinterpret_cast<const float4 *>(s0 + state_base + (size_t)i * DK + j);
+        Sr[j] = x.x; Sr[j + 1] = x.y; Sr[j + 2] = x.z; Sr[j + 3] = x.w;
+      }
+    } else {
 #pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16x2(S[2 * c], S[2 * c + 1]);
-      tmem_st32(taddr(tm, 32 * q4, TA0 + 64 * buf + 32 * hh), pk);
-      tmem_st_wait();
-      tc_fence_before();
+      for (int j = 0; j < NS; ++j) Sr[j] = 0.f;
+    }
+    auto write_operand = [&](int b) {  // row i of S in bf16 -> MN-major B operand
+      unsigned char *sb = sm + Cfg::OFF_SB + b * Cfg::SB_BYTES;
+#pragma unroll
+      for (int ch = 0; ch < NS / 8; ++ch) {
+        float x[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) x[e] = Sr[8 * ch + e];
+        st16(sb + sop_off<NS>(i, ch), pack8(x));
+      }
+      fence_async_smem();
     };
     if (nch > 0) {
       write_operand(0);
-      mbar_arrive(&op_ready[0]);
+      mbar_arrive(&sb_ready[0]);
     }
     for (int u = 0; u < nch; ++u) {
-      const int st = u % NSTAGE;
-      mbar_wait(bar_s, u & 1, err, KDA_DEVICE_TIMEOUT);
+      const int st = u % S;
+      if (!mbar_wait(ds_full, u & 1, err, KDA_DEVICE_TIMEOUT)) break;
       tc_fence_after();
-      float v[32];
-      const unsigned char *qc = sm + st * ST_BYTES + ST_QC;
-      mbar_wait(&full[st], (u / NSTAGE) & 1, err, KDA_DEVICE_TIMEOUT);
+      float v[NS];
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        tmem_ld32(taddr(tm, 32 * q4, TD_S + 64 * hh + 32 * part), v);
+      for (int p = 0; p < NS / 32; ++p) {
+        float w32[32];
+        tmem_ld32(taddr(tm, 32 * warp, Cfg::TD_S + 32 * p), w32);
         tmem_ld_wait();
 #pragma unroll
-        for (int seg = 0; seg < 4; ++seg) {
-          const uint4 w = *reinterpret_cast<const uint4 *>(
-              qc + rowimg_off(j, DK * 2, 8 * hh + 4 * part + seg));
+        for (int e = 0; e < 32; ++e) v[32 * p + e] = w32[e];
+      }
+      tc_fence_before();
+      if (!mbar_wait(&full[st], (u / S) & 1, err, KDA_DEVICE_TIMEOUT)) break;
+      const unsigned char *qc = sm + st * Cfg::ST_BYTES + Cfg::ST_QC;
+#pragma unroll
+      for (int p = 0; p < NS / 32; ++p) {
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(qc + p * QC_SLICE_BYTES + slice_off(i, ch));
           const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            S[32 * part + 8 * seg + 2 * e] = v[8 * seg + 2 * e] + bf16_lo(ww[e]);
-            S[32 * part + 8 * seg + 2 * e + 1] = v[8 * seg + 2 * e + 1] + bf16_hi(ww[e]);
+            const int j = 32 * p + 8 * ch + 2 * e;
+            Sr[j] = v[j] + bf16_lo(ww[e]);
+            Sr[j + 1] = v[j + 1] + bf16_hi(ww[e]);
           }
         }
       }
       if (u + 1 < nch) {
-        write_operand((u + 1) % 3);
-        mbar_arrive(&op_ready[(u + 1) % 3]);
-      } else {
-        tc_fence_before();
+        write_operand((u + 1) & 1);
+        mbar_arrive(&sb_ready[(u + 1) & 1]);
       }
       mbar_arrive(&empty[st]);
     }
     if (sT) {
 #pragma unroll
-      for (int r = 0; r < 64; ++r) sT[state_base + (size_t)(64 * hh + r) * DK + j] = S[r];
+      for (int j = 0; j < NS; j += 4)
+        *reinterpret_cast<float4 *>(sT + state_base + (size_t)i * DK + j) =
+            make_float4(Sr[j], Sr[j + 1], Sr[j + 2], Sr[j + 3]);
     }
-  } else if (warp < kChainWarps + kOutWarps) {
-    // ---------------- outputs: o = Q' S + O_intra ----------------
-    const int q4 = warp & 3;
-    const int j = 32 * q4 + lane;
-    const int otid = tid - 32 * kChainWarps;  // 0..127
-    __nv_bfloat16 *tile = reinterpret_cast<__nv_bfloat16 *>(sm + SC_OT);
+  } else if (warp < 6) {
+    // ---------------- outputs: row t of o = Q' S + O_intra ----------------
+    const int t = 32 * (warp - 4) + lane;  // TMEM lane quarter warp % 4 = warp - 4
     ChunkEntry ce = nch > 0 ? tab[c_begin] : ChunkEntry{0, 0, 0, 0};
     for (int u = 0; u < nch; ++u) {
-      const int st = u % NSTAGE;
+      const int st = u % S, b = u & 1;
       const ChunkEntry ce_next = (u + 1 < nch) ? tab[c_begin + u + 1] : ce;
-      mbar_wait(&bar_o[u & 1], (u >> 1) & 1, err, KDA_DEVICE_TIMEOUT);
+      if (!mbar_wait(&do_full[b], (u >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
       tc_fence_after();
-      mbar_wait(&full[st], (u / NSTAGE) & 1, err, KDA_DEVICE_TIMEOUT);
-      const unsigned char *oi = sm + st * ST_BYTES + ST_OI;
+      float v[NS];
 #pragma unroll
-      for (int part = 0; part < 2; ++part) {
-        float v[32];
-        tmem_ld32(taddr(tm, 32 * q4, TD_O + 64 * (u & 1) + 32 * part), v);
+      for (int p = 0; p < NS / 32; ++p) {
+        float w32[32];
+        tmem_ld32(taddr(tm, 32 * (warp - 4), Cfg::TD_O + NS * b + 32 * p), w32);
         tmem_ld_wait();
 #pragma unroll
-        for (int seg = 0; seg < 4; ++seg) {
-          const uint4 w =
-              *reinterpret_cast<const uint4 *>(oi + rowimg_off(j, C * 2, 4 * part + seg));
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int t = 32 * part + 8 * seg + 2 * e;
-            tile[t * DK + j] = __float2bfloat16_rn(v[8 * seg + 2 * e] + bf16_lo(ww[e]));
-            tile[(t + 1) * DK + j] = __float2bfloat16_rn(v[8 * seg + 2 * e + 1] + bf16_hi(ww[e]));
-          }
-        }
+        for (int e = 0; e < 32; ++e) v[32 * p + e] = w32[e];
       }
       tc_fence_before();
-      mbar_arrive(&o_free[u & 1]);
-      mbar_arrive(&empty[st]);
-      asm volatile("bar.sync %0, %1;" ::"n"(kOutBarrier), "n"(32 * kOutWarps) : "memory");
-      // tile rows t < len -> o[(start + t), h, :]  (16-byte stores, 256 B per row)
-      for (int item = otid; item < C * 16; item += 32 * kOutWarps) {
-        const int t = item >> 4, c8 = (item & 15) * 8;
-        if (t < ce.len)
-          *reinterpret_cast<uint4 *>(o + ((size_t)(ce.start + t) * H_v + h) * DK + c8) =
-              *reinterpret_cast<const uint4 *>(tile + t * DK + c8);
+      mbar_arrive(&do_free[b]);
+      if (!mbar_wait(&full[st], (u / S) & 1, err, KDA_DEVICE_TIMEOUT)) break;
+      const unsigned char *oi = sm + st * Cfg::ST_BYTES + Cfg::ST_OI;
+      uint4 out[NS / 8];
+#pragma unroll
+      for (int p = 0; p < NS / 32; ++p) {
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const uint4 w = *reinterpret_cast<const uint4 *>(oi + p * OI_SLICE_BYTES + slice_off(t, ch));
+          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+          float x[8];
+#pragma unroll
+          for (int e = 0; e < 4; ++e) {
+            x[2 * e] = v[32 * p + 8 * ch + 2 * e] + bf16_lo(ww[e]);
+            x[2 * e + 1] = v[32 * p + 8 * ch + 2 * e + 1] + bf16_hi(ww[e]);
+          }
+          out[4 * p + ch] = pack8(x);
+        }
       }
-      asm volatile("bar.sync %0, %1;" ::"n"(kOutBarrier), "n"(32 * kOutWarps) : "memory");
+      mbar_arrive(&empty[st]);
+      if (t < ce.len) {
+        uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(ce.start + t) * H_v + h) * DK + sl * NS);
+#pragma unroll
+        for (int q = 0; q < NS / 8; ++q) dst[q] = out[q];
+      }
       ce = ce_next;
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 0) tmem_dealloc(tm, 512);
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tm, Cfg::TMEM_COLS);
 }
-
 // ---------------------------------------------------------------------------
 // host side
 // ---------------------------------------------------------------------------
@@ -1171,6 +1253,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
   unsigned char *ws = static_cast<unsigned char *>(a.workspace);
   int32_t *hdr = reinterpret_cast<int32_t *>(ws);
   int32_t *seq_off = reinterpret_cast<int32_t *>(ws + L.seq_off);
+  int32_t *order = reinterpret_cast<int32_t *>(ws + L.order);
   ChunkEntry *tab = reinterpret_cast<ChunkEntry *>(ws + L.tab);
   unsigned char *slots = ws + L.slots;
   const int64_t max_chunks = T_total / C + a.num_seqs;
@@ -1194,7 +1277,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
   {
     TraceScope tr("plan_kernel", stream);
     plan_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, a.num_seqs, a.T, (int)T_total, hdr,
-                                        seq_off, tab);
+                                        seq_off, order, tab);
   }
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1214,13 +1297,19 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
 
-  e = cudaFuncSetAttribute(chunk_scan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, SCAN_SMEM);
+  // Four 32-column slices per chain while they fit on the SMs in one wave,
+  // else two 64-column slices (twice the work per CTA, half the re-reads of P, Q').
+  const int64_t chains = (int64_t)a.num_seqs * a.H_v;
+  const bool narrow = chains * 4 <= sm_count();
+  auto scan = narrow ? chunk_scan_kernel<32> : chunk_scan_kernel<64>;
+  const uint32_t scan_smem = narrow ? ScanCfg<32>::SMEM : ScanCfg<64>::SMEM;
+  e = cudaFuncSetAttribute(scan, cudaFuncAttributeMaxDynamicSharedMemorySize, scan_smem);
   if (e != cudaSuccess) return e;
-  dim3 gs((unsigned)a.num_seqs, (unsigned)a.H_v);
+  dim3 gs((unsigned)(chains * (narrow ? 4 : 2)));
   {
     TraceScope tr("chunk_scan_kernel", stream);
-    chunk_scan_kernel<<<gs, kScanThreads, SCAN_SMEM, stream>>>(
-        hdr, seq_off, tab, slots, (__nv_bfloat16 *)a.o, a.initial_state, a.final_state,
+    scan<<<gs, kScanThreads, scan_smem, stream>>>(
+        hdr, seq_off, order, tab, slots, (__nv_bfloat16 *)a.o, a.initial_state, a.final_state,
         a.state_slots, a.num_slots, a.H_v, hdr);
   }
   return cudaGetLastError();

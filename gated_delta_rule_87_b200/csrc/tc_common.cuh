@@ -227,18 +227,30 @@ __device__ __forceinline__ uint32_t sw128(uint32_t byte_off) {
   return byte_off ^ (((byte_off >> 7) & 7u) << 4);
 }
 
+// 64-byte swizzle: within every 512-byte atom of 8 rows x 64 bytes, the
+// 16-byte chunk index (address bits 4..5) is XORed with bits 7..8.  Atoms
+// must be 512-byte aligned.
+__device__ __forceinline__ uint32_t sw64(uint32_t byte_off) {
+  return byte_off ^ (((byte_off >> 7) & 3u) << 4);
+}
+
 // Descriptor fields: start address >> 4 (bits 0..13), leading byte offset >> 4
 // (16..29), stride byte offset >> 4 (32..45), version 1 (bit 46), base offset 0,
-// layout type SWIZZLE_128B = 2 (bits 61..63).
-__device__ __forceinline__ uint64_t make_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
-                                                    uint32_t sbo_bytes) {
+// layout type in bits 61..63 (SWIZZLE_128B = 2, SWIZZLE_64B = 4).
+constexpr uint32_t kLayoutSw128 = 2, kLayoutSw64 = 4;
+__device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo_bytes,
+                                              uint32_t sbo_bytes, uint32_t layout) {
   uint64_t d = 0;
   d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
   d |= (uint64_t)((lbo_bytes >> 4) & 0x3FFFu) << 16;
   d |= (uint64_t)((sbo_bytes >> 4) & 0x3FFFu) << 32;
   d |= (uint64_t)1 << 46;
-  d |= (uint64_t)2 << 61;
+  d |= (uint64_t)layout << 61;
   return d;
+}
+__device__ __forceinline__ uint64_t make_desc_sw128(uint32_t saddr, uint32_t lbo_bytes,
+                                                    uint32_t sbo_bytes) {
+  return make_desc(saddr, lbo_bytes, sbo_bytes, kLayoutSw128);
 }
 
 // Instruction descriptor, kind::f16 with bf16 A and B, fp32 accumulator.
@@ -310,6 +322,13 @@ __device__ __forceinline__ uint32_t mnmajor_off(int k, int m, uint32_t mn_block_
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile_saddr, int k0,
                                                  uint32_t mn_block_bytes) {
   return make_desc_sw128(tile_saddr + (uint32_t)k0 * 128, mn_block_bytes, 1024);
+}
+
+// MN-major SW64 tile of exactly 32 MN-elements: K rows of 64 bytes, element
+// (k, m) at sw64(k * 64 + m * 2).  Descriptor for K rows [k0, k0 + 16) (one
+// MN atom, so the leading byte offset is unused).
+__device__ __forceinline__ uint64_t desc_mnmajor32(uint32_t tile_saddr, int k0) {
+  return make_desc(tile_saddr + (uint32_t)k0 * 64, 512, 512, kLayoutSw64);
 }
 
 }  // namespace tc
