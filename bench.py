@@ -382,12 +382,13 @@ def run_ours(args, world, rank, local):
 
 
 def gdr_launches_per_call(w: W.Workload, varlen: bool) -> int:
-    """Our kernels per prefill call.  Tensor-core path (bf16, d = 128): plan,
-    prep and scan.  fp32 path: the chunk kernel, plus the cu_seqlens check for
-    packed batches.  (The status reset is a memset, not a kernel.)"""
+    """Our kernels per prefill call.  Tensor-core path (bf16, d = 128): prep and
+    scan, plus the planning kernel for packed batches.  fp32 path: the chunk
+    kernel, plus the cu_seqlens check for packed batches.  (The status reset is
+    a memset, not a kernel.)"""
     tc = w.io_dtype == "bf16" and w.d_k == 128 and w.d_v == 128
     if tc:
-        return 3
+        return 3 if varlen else 2
     return 1 + (1 if varlen else 0)
 
 

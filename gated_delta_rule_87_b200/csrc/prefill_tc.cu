@@ -90,6 +90,29 @@ WsLayout ws_layout(int64_t T_total, int num_seqs) {
   return L;
 }
 
+// Where a kernel finds its chunks: for a dense batch (B sequences of T tokens)
+// they follow from the chunk index; for packed sequences from the planning
+// kernel's table, per-sequence offsets and scan order.
+struct Chunks {
+  const ChunkEntry *tab;
+  const int32_t *seq_off, *order;
+  int dense_T;  // > 0: dense batch of sequences of this length (no table)
+  int per_seq;  // dense: chunks per sequence
+  __device__ __forceinline__ ChunkEntry entry(int ck) const {
+    if (dense_T > 0) {
+      const int n = ck / per_seq, j = ck - n * per_seq;
+      return ChunkEntry{n, n * dense_T + j * C, min(C, dense_T - j * C), 0};
+    }
+    return tab[ck];
+  }
+  __device__ __forceinline__ int first(int n) const { return dense_T > 0 ? n * per_seq : seq_off[n]; }
+  __device__ __forceinline__ int seq(int r) const { return dense_T > 0 ? r : order[r]; }
+  // total chunks: dense from the shape, packed from the plan's header word
+  __device__ __forceinline__ int total(const int32_t *hdr, int num_seqs) const {
+    return dense_T > 0 ? num_seqs * per_seq : hdr[1];
+  }
+};
+
 // ---------------------------------------------------------------------------
 // planning: chunk table, per-sequence chunk offsets and the order in which
 // the scan takes the sequences (also validates cu_seqlens)
@@ -316,7 +339,7 @@ __global__ void __launch_bounds__(kPrepThreads, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                   const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_g,
                   const float *__restrict__ g_scalar, const float *__restrict__ beta, int H_qk,
-                  int H_v, int32_t *hdr, const ChunkEntry *__restrict__ tab,
+                  int H_v, int32_t *hdr, const Chunks chunks, int num_seqs,
                   unsigned char *__restrict__ slots) {
   extern __shared__ unsigned char smem_raw[];
   // 1024-byte aligned base, derived by pointer arithmetic on the shared array so
@@ -338,7 +361,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // persistent: this CTA walks (chunk, v-head) work items blockIdx.x,
   // blockIdx.x + gridDim.x, ...; the next item's tiles are loaded while the
   // current one finishes.
-  const int total = hdr[1] * H_v;
+  const int total = chunks.total(hdr, num_seqs) * H_v;
   int work = blockIdx.x;
   if (work >= total) return;
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -360,7 +383,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // ---- 1. TMA loads of an item's q, k, v (bf16, swizzled) and g (fp32) ----
   // Items' chunk-table entries are read one item ahead of their use, so no
   // thread waits on a global load between phases.
-  auto entry = [&](int w) { return w < total ? tab[w / H_v] : ChunkEntry{0, 0, 0, 0}; };
+  auto entry = [&](int w) { return w < total ? chunks.entry(w / H_v) : ChunkEntry{0, 0, 0, 0}; };
   auto issue_loads = [&](int w, const ChunkEntry &e) {  // thread 0
     const int ck = w / H_v, hh = w - ck * H_v, hkk = hh / (H_v / H_qk);
     const int ts = e.start;
@@ -965,9 +988,7 @@ __device__ __forceinline__ uint64_t sop_desc(uint32_t base, int kk) {
 
 template <int NS>
 __global__ void __launch_bounds__(kScanThreads, 1)
-chunk_scan_kernel(const int32_t *hdr, const int32_t *__restrict__ seq_off,
-                  const int32_t *__restrict__ order, const ChunkEntry *__restrict__ tab,
-                  const unsigned char *__restrict__ slots, __nv_bfloat16 *__restrict__ o,
+chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *__restrict__ slots, __nv_bfloat16 *__restrict__ o,
                   const float *s0, float *sT, const int32_t *__restrict__ state_slots,
                   int64_t num_slots, int H_v, int32_t *err) {
   using Cfg = ScanCfg<NS>;
@@ -987,9 +1008,9 @@ chunk_scan_kernel(const int32_t *hdr, const int32_t *__restrict__ seq_off,
   if (hdr[0] != KDA_DEVICE_OK) return;
   const int cid = blockIdx.x;
   const int sl = cid % NSL, h = (cid / NSL) % H_v;
-  const int n = order[cid / (NSL * H_v)];
+  const int n = chunks.seq(cid / (NSL * H_v));
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int c_begin = seq_off[n], nch = seq_off[n + 1] - c_begin;
+  const int c_begin = chunks.first(n), nch = chunks.first(n + 1) - c_begin;
 
   if (warp == 0) {
     tmem_alloc(tslot, Cfg::TMEM_COLS);
@@ -1059,8 +1080,8 @@ chunk_scan_kernel(const int32_t *hdr, const int32_t *__restrict__ seq_off,
       constexpr uint32_t idO = idesc_bf16(128, NS, true, true);   // Q' MN-major, S MN-major
       for (int u = 0; u < nch; ++u) {
         const int st = u % S, b = u & 1;
-        if (!mbar_wait(&sb_ready[b], (u >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
         if (!mbar_wait(&full[st], (u / S) & 1, err, KDA_DEVICE_TIMEOUT)) break;
+        if (!mbar_wait(&sb_ready[b], (u >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
         tc_fence_after();
         const uint32_t stage = smem_u32(sm + st * Cfg::ST_BYTES);
         const uint32_t sb = smem_u32(sm + Cfg::OFF_SB + b * Cfg::SB_BYTES);
@@ -1113,32 +1134,30 @@ chunk_scan_kernel(const int32_t *hdr, const int32_t *__restrict__ seq_off,
     }
     for (int u = 0; u < nch; ++u) {
       const int st = u % S;
+      // this chunk's Qc rows, read while the product runs
+      if (!mbar_wait(&full[st], (u / S) & 1, err, KDA_DEVICE_TIMEOUT)) break;
+      uint4 qv[NS / 8];
+      const unsigned char *qc = sm + st * Cfg::ST_BYTES + Cfg::ST_QC;
+#pragma unroll
+      for (int p = 0; p < NS / 32; ++p)
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch)
+          qv[4 * p + ch] = *reinterpret_cast<const uint4 *>(qc + p * QC_SLICE_BYTES + slice_off(i, ch));
       if (!mbar_wait(ds_full, u & 1, err, KDA_DEVICE_TIMEOUT)) break;
       tc_fence_after();
       float v[NS];
 #pragma unroll
-      for (int p = 0; p < NS / 32; ++p) {
-        float w32[32];
-        tmem_ld32(taddr(tm, 32 * warp, Cfg::TD_S + 32 * p), w32);
-        tmem_ld_wait();
-#pragma unroll
-        for (int e = 0; e < 32; ++e) v[32 * p + e] = w32[e];
-      }
+      for (int p = 0; p < NS / 32; ++p)
+        tmem_ld32(taddr(tm, 32 * warp, Cfg::TD_S + 32 * p), *reinterpret_cast<float(*)[32]>(&v[32 * p]));
+      tmem_ld_wait();
       tc_fence_before();
-      if (!mbar_wait(&full[st], (u / S) & 1, err, KDA_DEVICE_TIMEOUT)) break;
-      const unsigned char *qc = sm + st * Cfg::ST_BYTES + Cfg::ST_QC;
 #pragma unroll
-      for (int p = 0; p < NS / 32; ++p) {
+      for (int c8 = 0; c8 < NS / 8; ++c8) {
+        const uint32_t ww[4] = {qv[c8].x, qv[c8].y, qv[c8].z, qv[c8].w};
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const uint4 w = *reinterpret_cast<const uint4 *>(qc + p * QC_SLICE_BYTES + slice_off(i, ch));
-          const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            const int j = 32 * p + 8 * ch + 2 * e;
-            Sr[j] = v[j] + bf16_lo(ww[e]);
-            Sr[j + 1] = v[j + 1] + bf16_hi(ww[e]);
-          }
+        for (int e = 0; e < 4; ++e) {
+          Sr[8 * c8 + 2 * e] = v[8 * c8 + 2 * e] + bf16_lo(ww[e]);
+          Sr[8 * c8 + 2 * e + 1] = v[8 * c8 + 2 * e + 1] + bf16_hi(ww[e]);
         }
       }
       if (u + 1 < nch) {
@@ -1156,10 +1175,10 @@ chunk_scan_kernel(const int32_t *hdr, const int32_t *__restrict__ seq_off,
   } else if (warp < 6) {
     // ---------------- outputs: row t of o = Q' S + O_intra ----------------
     const int t = 32 * (warp - 4) + lane;  // TMEM lane quarter warp % 4 = warp - 4
-    ChunkEntry ce = nch > 0 ? tab[c_begin] : ChunkEntry{0, 0, 0, 0};
+    ChunkEntry ce = nch > 0 ? chunks.entry(c_begin) : ChunkEntry{0, 0, 0, 0};
     for (int u = 0; u < nch; ++u) {
       const int st = u % S, b = u & 1;
-      const ChunkEntry ce_next = (u + 1 < nch) ? tab[c_begin + u + 1] : ce;
+      const ChunkEntry ce_next = (u + 1 < nch) ? chunks.entry(c_begin + u + 1) : ce;
       if (!mbar_wait(&do_full[b], (u >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
       tc_fence_after();
       float v[NS];
@@ -1274,25 +1293,32 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
     mg = mv;  // unused
   }
 
-  {
+  // a dense batch needs no planning: its chunks follow from the shape
+  Chunks chunks{tab, seq_off, order, 0, 0};
+  cudaError_t e = cudaSuccess;
+  if (a.cu_seqlens) {
     TraceScope tr("plan_kernel", stream);
     plan_kernel<<<1, 1024, 0, stream>>>(a.cu_seqlens, a.num_seqs, a.T, (int)T_total, hdr,
                                         seq_off, order, tab);
+    e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+  } else {
+    chunks.dense_T = a.T;
+    chunks.per_seq = (a.T + C - 1) / C;
   }
-  cudaError_t e = cudaGetLastError();
-  if (e != cudaSuccess) return e;
 
   auto prep = !a.channel_gate ? chunk_prep_kernel<false, false>
                : a.decay_first ? chunk_prep_kernel<true, true>
                                : chunk_prep_kernel<true, false>;
   e = cudaFuncSetAttribute(prep, cudaFuncAttributeMaxDynamicSharedMemorySize, PREP_SMEM);
   if (e != cudaSuccess) return e;
-  const int64_t items = max_chunks * a.H_v;
+  const int64_t items = (a.cu_seqlens ? max_chunks : (int64_t)a.num_seqs * chunks.per_seq) * a.H_v;
   dim3 gp((unsigned)(items < sm_count() ? items : sm_count()));
   {
     TraceScope tr("chunk_prep_kernel", stream);
     prep<<<gp, kPrepThreads, PREP_SMEM, stream>>>(mq, mk, mv, mg, a.channel_gate ? nullptr : a.g,
-                                                 a.beta, a.H_qk, a.H_v, hdr, tab, slots);
+                                                 a.beta, a.H_qk, a.H_v, hdr, chunks, a.num_seqs,
+                                                 slots);
   }
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
@@ -1309,7 +1335,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
   {
     TraceScope tr("chunk_scan_kernel", stream);
     scan<<<gs, kScanThreads, scan_smem, stream>>>(
-        hdr, seq_off, order, tab, slots, (__nv_bfloat16 *)a.o, a.initial_state, a.final_state,
+        hdr, chunks, slots, (__nv_bfloat16 *)a.o, a.initial_state, a.final_state,
         a.state_slots, a.num_slots, a.H_v, hdr);
   }
   return cudaGetLastError();

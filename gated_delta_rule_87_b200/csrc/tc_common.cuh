@@ -61,6 +61,20 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   return ok != 0;
 }
 
+// Non-blocking test of the phase with the given parity (no suspend: cheaper
+// than try_wait when the phase has usually completed already).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
 // Upper bound on polls of one mbarrier phase (about kMaxPolls x 1 ms, i.e.
 // seconds): far above any legitimate wait, but a wait that can never finish
 // still ends.
@@ -71,6 +85,7 @@ constexpr uint32_t kMaxPolls = 4096;
 // remaining work instead of hanging.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *err,
                                           int32_t code) {
+  if (mbar_test_wait(bar, parity)) return true;
   for (uint32_t i = 0; i < kMaxPolls; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   if (err) atomicExch(err, code);
