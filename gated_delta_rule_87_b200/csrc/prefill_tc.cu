@@ -236,11 +236,9 @@ constexpr uint32_t OFF_KAB = OFF_G, OFF_KBB = OFF_G + 16384;
 
 // X region, gram phase
 constexpr uint32_t X_R = 0;           // 32 KB, K-major B [128 rows][128], blocks 16 KB apart
-constexpr uint32_t X_LEFT = 32768;    // 80 KB, four overlapped K-major A tiles
-constexpr uint32_t LEFT_BLOCK = 40960;
-__device__ __forceinline__ uint32_t left_off(int J) {
-  return J == 0 ? 0u : (J == 1 ? 12288u : (J == 2 ? 20480u : 24576u));
-}
+constexpr uint32_t X_LEFT = 32768;    // 48 KB, two overlapped K-major A tiles (anchors E_0, E_2)
+constexpr uint32_t LEFT_BLOCK = 24576;  // 64-column blocks of the left tiles
+constexpr uint32_t LEFT_G1 = 8192;      // anchor-E_2 tile: its rows 64..127 land past the E_0 tile's
 // X region, after the Gram MMAs
 constexpr uint32_t X_AWBW = 0;        // 16 KB K-major B [128 i'][64 j]
 constexpr uint32_t X_BE = 16384;      // 8 KB  K-major B [64 i][64 j]
@@ -372,7 +370,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   if (tid == 0) {
     mbar_init(bar_tma, 1);
-    mbar_init(bar_mma, 1);
+    mbar_init(bar_mma, 2);  // every product round: one commit from each issuing thread
     mbar_fence_init();
   }
   tc_fence_before();
@@ -499,7 +497,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   // ---- 3. one pass builds every operand of the chunk ----
   {
-    float F0[4], F1[4];  // e^{E_{I-1} - E_J}: J < I products (<= 1), J = I e^{-sum g} (>= 1)
+    // Gram anchors E_0 (key sub-chunks 0, 1) and E_2 (2, 3).  Row factors
+    // F_A = e^{E_{I-1} - E_A} for a row of sub-chunk I >= A: 1/PB_A >= 1 for
+    // I = A, 1 for I = A + 1, products of PB <= 1 beyond; a key of sub-chunk
+    // J = A + 1 takes e^{E_A - E_J} = 1/PB_J on top of its suffix product.
     float ei0 = 1.f, ei1 = 1.f, ge0 = 1.f, ge1 = 1.f;  // e^{E_{I-1}}, e^{G_L - E_I}
 #pragma unroll
     for (int J = 0; J < 4; ++J) {
@@ -512,23 +513,21 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         ge1 *= sPblk[J * DK + c2 + 1];
       }
     }
-#pragma unroll
-    for (int J = 0; J < 4; ++J) {
-      float f0 = 1.f, f1 = 1.f;
-      if (J < bI) {
-#pragma unroll
-        for (int J2 = 0; J2 < 4; ++J2)
-          if (J2 > J && J2 < bI) {
-            f0 *= sPblk[J2 * DK + c2];
-            f1 *= sPblk[J2 * DK + c2 + 1];
-          }
-      } else if (J == bI) {
-        f0 = expf(-sGsum[bI * DK + c2]);
-        f1 = expf(-sGsum[bI * DK + c2 + 1]);
+    const float inv0 = expf(-sGsum[bI * DK + c2]), inv1 = expf(-sGsum[bI * DK + c2 + 1]);  // 1/PB_I
+    float fa0 = 1.f, fa1 = 1.f;  // anchor E_0
+    if (bI == 0) {
+      fa0 = inv0;
+      fa1 = inv1;
+    } else if (bI >= 2) {
+      fa0 = sPblk[1 * DK + c2];
+      fa1 = sPblk[1 * DK + c2 + 1];
+      if (bI == 3) {
+        fa0 *= sPblk[2 * DK + c2];
+        fa1 *= sPblk[2 * DK + c2 + 1];
       }
-      F0[J] = f0;
-      F1[J] = f1;
     }
+    const float fb0 = bI == 2 ? inv0 : 1.f, fb1 = bI == 2 ? inv1 : 1.f;  // anchor E_2
+    const float rf0 = (bI & 1) ? inv0 : 1.f, rf1 = (bI & 1) ? inv1 : 1.f;  // key side
     if (bI == 0 && rh == 0) {
       sGLe[c2] = ge0 * sPblk[c2];  // e^{G_L}: product over all four sub-chunks
       sGLe[c2 + 1] = ge1 * sPblk[c2 + 1];
@@ -562,19 +561,24 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       pq0 = bq0;
       pq1 = bq1;
       const int rowK = 32 * bI + 8 * rh + r, rowQ = rowK + 16;
-      // Gram right operand (keys scaled to their sub-chunk end)
+      // Gram right operand (keys scaled to their group's anchor)
       const uint32_t rb = X_R + (c2 >> 6) * 16384;
-      *reinterpret_cast<uint32_t *>(sX + rb + kmajor_off(rowK, c2 & 63)) = pack_bf16x2(k0 * rw0, k1 * rw1);
-      *reinterpret_cast<uint32_t *>(sX + rb + kmajor_off(rowQ, c2 & 63)) = pack_bf16x2(k0 * re0, k1 * re1);
-      // Gram left operands, one per key sub-chunk J <= I
-#pragma unroll
-      for (int J = 0; J < 4; ++J) {
-        if (J <= bI) {
-          const uint32_t lb = X_LEFT + left_off(J) + (c2 >> 6) * LEFT_BLOCK;
-          *reinterpret_cast<uint32_t *>(sX + lb + kmajor_off(rowK, c2 & 63)) =
-              pack_bf16x2(k0 * bk0 * F0[J], k1 * bk1 * F1[J]);
-          *reinterpret_cast<uint32_t *>(sX + lb + kmajor_off(rowQ, c2 & 63)) =
-              pack_bf16x2(q0 * bq0 * F0[J], q1 * bq1 * F1[J]);
+      *reinterpret_cast<uint32_t *>(sX + rb + kmajor_off(rowK, c2 & 63)) =
+          pack_bf16x2(k0 * rw0 * rf0, k1 * rw1 * rf1);
+      *reinterpret_cast<uint32_t *>(sX + rb + kmajor_off(rowQ, c2 & 63)) =
+          pack_bf16x2(k0 * re0 * rf0, k1 * re1 * rf1);
+      // Gram left operands: anchor E_0 (all rows), anchor E_2 (sub-chunks 2, 3)
+      {
+        const uint32_t lb = X_LEFT + (c2 >> 6) * LEFT_BLOCK;
+        *reinterpret_cast<uint32_t *>(sX + lb + kmajor_off(rowK, c2 & 63)) =
+            pack_bf16x2(k0 * bk0 * fa0, k1 * bk1 * fa1);
+        *reinterpret_cast<uint32_t *>(sX + lb + kmajor_off(rowQ, c2 & 63)) =
+            pack_bf16x2(q0 * bq0 * fa0, q1 * bq1 * fa1);
+        if (bI >= 2) {
+          *reinterpret_cast<uint32_t *>(sX + lb + LEFT_G1 + kmajor_off(rowK, c2 & 63)) =
+              pack_bf16x2(k0 * bk0 * fb0, k1 * bk1 * fb1);
+          *reinterpret_cast<uint32_t *>(sX + lb + LEFT_G1 + kmajor_off(rowQ, c2 & 63)) =
+              pack_bf16x2(q0 * bq0 * fb0, q1 * bq1 * fb1);
         }
       }
       // K e^{Gp} over k, q e^{G} over q (same element, same owner), beta K e^{G_L - G|Gp}
@@ -591,18 +595,17 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
   tc_fence_after();
 
-  // ---- 4. Gram MMAs: for each key sub-chunk J, [K;Q] rows x 32 key columns ----
-  if (tid == 0) {
-    constexpr uint32_t ID = idesc_bf16(128, 32, false, false);
-    const uint32_t r_base = smem_u32(sX + X_R);
+  // ---- 4. Gram MMAs: per anchor group A, [K;Q] rows x 64 key columns (w, e of
+  //         two key sub-chunks); one issuing thread per group ----
+  if (tid == 0 || tid == 32) {
+    const int A = tid >> 5;
+    constexpr uint32_t ID = idesc_bf16(128, 64, false, false);
+    const uint32_t a_base = smem_u32(sX + X_LEFT + A * LEFT_G1);
+    const uint32_t r_base = smem_u32(sX + X_R + A * 8192);
 #pragma unroll
-    for (int J = 0; J < 4; ++J) {
-      const uint32_t a_base = smem_u32(sX + X_LEFT + left_off(J));
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        mma_bf16(tm + TM_GRAM + 32 * J, desc_kmajor(a_base, 16 * kk, LEFT_BLOCK),
-                 desc_kmajor(r_base + 4096 * J, 16 * kk, 16384), ID, kk > 0);
-    }
+    for (int kk = 0; kk < 8; ++kk)
+      mma_bf16(tm + TM_GRAM + 64 * A, desc_kmajor(a_base, 16 * kk, LEFT_BLOCK),
+               desc_kmajor(r_base, 16 * kk, 16384), ID, kk > 0);
     mma_commit(bar_mma);
   }
   __syncwarp();
@@ -746,6 +749,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_W, desc_mnmajor(smem_u32(sK), 16 * kk, 8192),
                desc_kmajor(tinvb, 16 * kk, 0), idesc_bf16(128, 64, true, false), kk > 0);
+    mma_commit(bar_mma);
+  } else if (tid == 32) {
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_Y, desc_mnmajor(smem_u32(sV), 16 * kk, 8192),
@@ -787,21 +792,24 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const uint32_t tinvb = smem_u32(sX + X_TINVB), wsm = smem_u32(sX + X_W);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tm + TM_U, desc_kmajor(smem_u32(sX + X_Y), 16 * kk, 0), desc_kmajor(tinvb, 16 * kk, 0),
+               idesc_bf16(128, 64, false, false), kk > 0);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tm + TM_X, desc_kmajor(wsm, 16 * kk, 0), desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0),
+               idesc_bf16(128, 64, false, false), kk > 0);
+    mma_commit(bar_mma);
+  } else if (tid == 32) {
+    const uint32_t wsm = smem_u32(sX + X_W);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_OI, desc_kmajor(smem_u32(sX + X_AWBW + 64 * 128), 16 * kk, 0),
                desc_mnmajor(smem_u32(sV), 16 * kk, 8192), idesc_bf16(128, 128, false, true),
                kk > 0);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_U, desc_kmajor(smem_u32(sX + X_Y), 16 * kk, 0), desc_kmajor(tinvb, 16 * kk, 0),
-               idesc_bf16(128, 64, false, false), kk > 0);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_P, desc_mnmajor(smem_u32(sm + OFF_KBB), 16 * kk, 8192), desc_kmajor(wsm, 16 * kk, 0),
                idesc_bf16(128, 128, true, false), kk > 0);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_X, desc_kmajor(wsm, 16 * kk, 0), desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0),
-               idesc_bf16(128, 64, false, false), kk > 0);
     mma_commit(bar_mma);
   }
   __syncwarp();
@@ -828,12 +836,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   // ---- 9. O_intra -= tril(B_e) beta U (M = 128 as in step 8);
   //         Qc = (beta K e^{G_L-G})^T V - (beta K e^{G_L-Gp})^T U: lanes i, columns j ----
-  if (tid == 0) {
+  if (tid == 32) {
     const uint32_t usm = smem_u32(sX + X_U);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_OI, desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0), desc_kmajor(usm, 16 * kk, 0),
                idesc_bf16(128, 128, false, false, true), 1);
+    mma_commit(bar_mma);
+  } else if (tid == 0) {
+    const uint32_t usm = smem_u32(sX + X_U);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sm + OFF_KAB), 16 * kk, 8192),
