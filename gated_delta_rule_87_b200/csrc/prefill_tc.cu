@@ -219,9 +219,11 @@ constexpr int kPrepThreads = 512;
 constexpr uint32_t OFF_Q = 0;         // q tile, two K-major SW128 [64 t][64 c] blocks; later q.e^{G}
 constexpr uint32_t OFF_K = 16384;     // k tile; later K.e^{Gp} (same bytes: MN-major [t][c])
 constexpr uint32_t OFF_V = 32768;     // v tile (MN-major operand, 64-wide blocks 8 KB apart)
-constexpr uint32_t OFF_G = 49152;     // g fp32 [64][128]; later beta K.e^{G_L-G} | beta K.e^{G_L-Gp}
-constexpr uint32_t OFF_X = 81920;     // 112 KB phase-dependent region
-constexpr uint32_t OFF_MISC = 196608;
+constexpr uint32_t OFF_KAB = 49152;   // beta K.e^{G_L-G}
+constexpr uint32_t OFF_KBB = 65536;   // beta K.e^{G_L-Gp}
+constexpr uint32_t OFF_G = 81920;     // g fp32 [64][128]; the next item's lands once the decays are taken
+constexpr uint32_t OFF_X = 114688;    // 96 KB phase-dependent region
+constexpr uint32_t OFF_MISC = 212992;
 constexpr uint32_t MISC_BETA = 0;      // f32[64]
 constexpr uint32_t MISC_GSC = 256;     // f32[64] scalar gate
 constexpr uint32_t MISC_PBLK = 512;    // f32[4][128] product of a over each sub-chunk
@@ -232,7 +234,6 @@ constexpr uint32_t MISC_TSLOT = 5136;  // u32
 constexpr uint32_t MISC_XP = 6144;     // f32[4][2][128] product of a over each half sub-chunk
 constexpr uint32_t MISC_XS = 10240;    // f32[4][2][128] sum of g over each half sub-chunk
 constexpr uint32_t PREP_SMEM = OFF_MISC + 14336 + 1024;
-constexpr uint32_t OFF_KAB = OFF_G, OFF_KBB = OFF_G + 16384;
 
 // X region, gram phase
 constexpr uint32_t X_R = 0;           // 32 KB, K-major B [128 rows][128], blocks 16 KB apart
@@ -252,10 +253,10 @@ constexpr uint32_t X_U = 65536;       // after T3: K-major [n][t]
 // slot images, staged in shared memory and bulk-copied to the workspace; the
 // copies' reads of these bytes only have to finish before the next item's
 // operand build
-constexpr uint32_t X_QPI = 0;         // after T4 issue: Q' image (16 KB)
-constexpr uint32_t X_PI = 81920;      // after T4 issue: P image (32 KB)
-constexpr uint32_t X_QCI = 16384;     // after T4: Qc image (32 KB)
-constexpr uint32_t X_OII = 49152;     // after T4: O_intra image (16 KB)
+constexpr uint32_t X_QPI = 0;         // written during the last products: Q' image (16 KB)
+constexpr uint32_t X_PI = 32768;      // written during the last products: P image (32 KB)
+constexpr uint32_t X_OII = 16384;     // after the last products: O_intra image (16 KB)
+constexpr uint32_t X_QCI = 65536;     // after the last products: Qc image (32 KB)
 
 // TMEM columns (W, Y die at their readback, U at its readback)
 constexpr uint32_t TM_GRAM = 0, TM_P = 0, TM_OI = 128, TM_W = 256, TM_Y = 320, TM_U = 256,
@@ -382,19 +383,27 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // Items' chunk-table entries are read one item ahead of their use, so no
   // thread waits on a global load between phases.
   auto entry = [&](int w) { return w < total ? chunks.entry(w / H_v) : ChunkEntry{0, 0, 0, 0}; };
-  auto issue_loads = [&](int w, const ChunkEntry &e) {  // thread 0
-    const int ck = w / H_v, hh = w - ck * H_v, hkk = hh / (H_v / H_qk);
+  // g is loaded as soon as the previous item has taken its decays (its bytes
+  // join the phase without an arrival); q, k and v when the previous item is
+  // done with them (the arrival).  Thread 0.
+  auto load_g = [&](int w, const ChunkEntry &e) {
+    if (CHANNEL) {
+      fence_async_smem();
+      mbar_expect_tx(bar_tma, 32768);
+      tma_load_3d(sG, &tm_g, 0, w % H_v, e.start, bar_tma);
+    }
+  };
+  auto load_qkv = [&](int w, const ChunkEntry &e) {
+    const int hh = w % H_v, hkk = hh / (H_v / H_qk);
     const int ts = e.start;
-    (void)ck;
     fence_async_smem();
-    mbar_arrive_expect_tx(bar_tma, 3 * 16384 + (CHANNEL ? 32768 : 0));
+    mbar_arrive_expect_tx(bar_tma, 3 * 16384);
 #pragma unroll
     for (int cb = 0; cb < 2; ++cb) {
       tma_load_3d(sQ + cb * 8192, &tm_q, cb * 64, hkk, ts, bar_tma);
       tma_load_3d(sK + cb * 8192, &tm_k, cb * 64, hkk, ts, bar_tma);
       tma_load_3d(sV + cb * 8192, &tm_v, cb * 64, hh, ts, bar_tma);
     }
-    if (CHANNEL) tma_load_3d(sG, &tm_g, 0, hh, ts, bar_tma);
   };
   auto prefetch_l2 = [&](int w, const ChunkEntry &e) {  // thread 0: a later item's tiles into L2
     const int ck = w / H_v, hh = w - ck * H_v, hkk = hh / (H_v / H_qk);
@@ -417,7 +426,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   float nbeta = 0.f, ngsc = 0.f;  // the coming item's, loaded one item ahead
   ChunkEntry ce = entry(work), ce_next = entry(work + gridDim.x);
   if (tid == 0) {
-    issue_loads(work, ce);
+    load_g(work, ce);
+    load_qkv(work, ce);
     if (work + (int)gridDim.x < total) prefetch_l2(work + gridDim.x, ce_next);
   }
   if (tid < C) load_beta(work, ce, nbeta, ngsc);
@@ -493,7 +503,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   // the previous item's image copies must have read the X region before it is rebuilt
   if (tid == 0) bulk_wait_read0();
-  __syncthreads();  // g is consumed: its region is reused below
+  __syncthreads();  // g is consumed: the next item's lands there
+  if (tid == 0 && next < total) {
+    load_g(next, ce_next);
+    if (next + (int)gridDim.x < total) prefetch_l2(next + gridDim.x, ce_next2);
+  }
 
   // ---- 3. one pass builds every operand of the chunk ----
   {
@@ -903,10 +917,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     bulk_commit();
   }
   // the input tiles are consumed: start the next item's loads now
-  if (tid == 0 && next < total) {
-    issue_loads(next, ce_next);
-    if (next + (int)gridDim.x < total) prefetch_l2(next + gridDim.x, ce_next2);
-  }
+  if (tid == 0 && next < total) load_qkv(next, ce_next);
   if (tid < C && next < total) load_beta(next, ce_next, nbeta, ngsc);
   {
     // warp (quad, qtr) holds rows 32 quad + lane, value columns 32 qtr .. +31,
