@@ -229,8 +229,8 @@ constexpr uint32_t MISC_GSC = 256;     // f32[64] scalar gate
 constexpr uint32_t MISC_PBLK = 512;    // f32[4][128] product of a over each sub-chunk
 constexpr uint32_t MISC_GSUM = 2560;   // f32[4][128] sum of g over each sub-chunk
 constexpr uint32_t MISC_GLE = 4608;    // f32[128] e^{G_L}
-constexpr uint32_t MISC_BAR = 5120;    // 2 x u64
-constexpr uint32_t MISC_TSLOT = 5136;  // u32
+constexpr uint32_t MISC_BAR = 5120;    // 5 x u64
+constexpr uint32_t MISC_TSLOT = 5160;  // u32
 constexpr uint32_t MISC_XP = 6144;     // f32[4][2][128] product of a over each half sub-chunk
 constexpr uint32_t MISC_XS = 10240;    // f32[4][2][128] sum of g over each half sub-chunk
 constexpr uint32_t PREP_SMEM = OFF_MISC + 14336 + 1024;
@@ -247,19 +247,22 @@ constexpr uint32_t X_TINVB = 24576;   // 8 KB  K-major B [64 i][64 j]; scratch b
 constexpr int LDN = 68;               // padded row stride (floats) of the fp32 64x64 tiles
 constexpr uint32_t X_NAE = 32768;     // 17 KB f32 [64][LDN]  (N = tril(A_e) diag(beta))
 constexpr uint32_t X_TINVF = 50176;   // 17 KB f32 [64][LDN]  (T^{-1}); both dead after step 6
-constexpr uint32_t X_W = 32768;       // after T2: K-major [c][t]
-constexpr uint32_t X_Y = 49152;       // after T2: K-major [n][t]
-constexpr uint32_t X_U = 65536;       // after T3: K-major [n][t]
+constexpr uint32_t X_Y = 69632;       // while T^{-1} is built: K-major [n][t]
+constexpr uint32_t X_W = 32768;       // after T^{-1}: K-major [c][t]
+constexpr uint32_t X_U = 49152;       // after T^{-1}: K-major [n][t]
 // slot images, staged in shared memory and bulk-copied to the workspace; the
 // copies' reads of these bytes only have to finish before the next item's
 // operand build
-constexpr uint32_t X_QPI = 0;         // written during the last products: Q' image (16 KB)
-constexpr uint32_t X_PI = 32768;      // written during the last products: P image (32 KB)
+constexpr uint32_t X_QPI = 0;         // after P and X: Q' image (16 KB)
+constexpr uint32_t X_PI = 65536;      // after P and X: P image (32 KB)
 constexpr uint32_t X_OII = 16384;     // after the last products: O_intra image (16 KB)
-constexpr uint32_t X_QCI = 65536;     // after the last products: Qc image (32 KB)
+constexpr uint32_t X_QCI = 32768;     // after the last products: Qc image (32 KB)
 
 // TMEM columns (W, Y die at their readback, U at its readback)
-constexpr uint32_t TM_GRAM = 0, TM_P = 0, TM_OI = 128, TM_W = 256, TM_Y = 320, TM_U = 256,
+// Rounds of products: the Gram; Y and the first O_intra term (issued before
+// T^{-1} is built, which needs neither); W and U; then P and X (one thread)
+// beside the second O_intra term and Qc (another).
+constexpr uint32_t TM_GRAM = 0, TM_Y = 320, TM_OI = 128, TM_W = 256, TM_U = 0, TM_P = 0,
                    TM_QC = 256, TM_X = 384;
 
 __device__ __forceinline__ float ld_bf16(const unsigned char *base, uint32_t off) {
@@ -353,7 +356,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   float *sGsum = reinterpret_cast<float *>(sm + OFF_MISC + MISC_GSUM);
   float *sGLe = reinterpret_cast<float *>(sm + OFF_MISC + MISC_GLE);
   uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + OFF_MISC + MISC_BAR);
-  uint64_t *bar_mma = bar_tma + 1;
+  uint64_t *bar_mma = bar_tma + 1;   // the Gram, then W and U (two commits each)
+  uint64_t *bar_yo = bar_tma + 2;    // Y and the first O_intra term (two commits)
+  uint64_t *bar_px = bar_tma + 3;    // P and X (one commit)
+  uint64_t *bar_oq = bar_tma + 4;    // the second O_intra term and Qc (one commit)
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + MISC_TSLOT);
 
   if (hdr[0] != KDA_DEVICE_OK) return;
@@ -371,7 +377,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   if (tid == 0) {
     mbar_init(bar_tma, 1);
-    mbar_init(bar_mma, 2);  // every product round: one commit from each issuing thread
+    mbar_init(bar_mma, 2);
+    mbar_init(bar_yo, 2);
+    mbar_init(bar_px, 1);
+    mbar_init(bar_oq, 1);
     mbar_fence_init();
   }
   tc_fence_before();
@@ -675,15 +684,36 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   __syncthreads();
 
-  // ---- 6. T^{-1}, T = I + N, N = tril_{-1}(A_e) diag(beta) (blocked, fp32) ----
-  // Unit lower triangular, so T^{-1} is built block by block:
-  //   diagonal 16x16 blocks by forward substitution (fp32, one thread per column);
-  //   T^{-1}[h][l] = -T^{-1}[h][h] N[h][l] T^{-1}[l][l] for the 16x16 blocks below
-  //   the diagonal pairs, then for the lower-left 32x32 block.  The block
-  //   products are warp-level tf32 MMAs with fp32 accumulation: too small for
-  //   the CTA-wide tensor-core path, and tf32 (10-bit mantissa) keeps them well
-  //   inside the bf16 rounding every T^{-1} entry gets afterwards.
-  {
+  // ---- 6. products that need no T^{-1}, issued before it is built:
+  //         Y^T = V^T (A_w beta)^T;  O_intra = tril(B_w) beta V (rows t < 64 of an
+  //         M = 128 product whose upper 64 rows read the bytes after the operand
+  //         and are discarded) ----
+  if (tid == 0) {
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tm + TM_Y, desc_mnmajor(smem_u32(sV), 16 * kk, 8192),
+               desc_kmajor(smem_u32(sX + X_AWBW), 16 * kk, 0), idesc_bf16(128, 64, true, false),
+               kk > 0);
+    mma_commit(bar_yo);
+  } else if (tid == 32) {
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tm + TM_OI, desc_kmajor(smem_u32(sX + X_AWBW + 64 * 128), 16 * kk, 0),
+               desc_mnmajor(smem_u32(sV), 16 * kk, 8192), idesc_bf16(128, 128, false, true),
+               kk > 0);
+    mma_commit(bar_yo);
+  }
+
+  if (warp < 8) {
+    // ---- 7. T^{-1}, T = I + N, N = tril_{-1}(A_e) diag(beta) (blocked, fp32), warps 0-7 ----
+    // Unit lower triangular, so T^{-1} is built block by block:
+    //   diagonal 16x16 blocks by forward substitution (fp32, one thread per column);
+    //   T^{-1}[h][l] = -T^{-1}[h][h] N[h][l] T^{-1}[l][l] for the 16x16 blocks below
+    //   the diagonal pairs, then for the lower-left 32x32 block.  The block
+    //   products are warp-level tf32 MMAs with fp32 accumulation: too small for
+    //   the CTA-wide tensor-core path, and tf32 (10-bit mantissa) keeps them well
+    //   inside the bf16 rounding every T^{-1} entry gets afterwards.
+    constexpr int kTinvBar = 2, kTinvThreads = 256;
     const float *nae = reinterpret_cast<const float *>(sX + X_NAE);
     float *tinv = reinterpret_cast<float *>(sX + X_TINVF);
     float *tmp = reinterpret_cast<float *>(sX + X_TINVB);  // fp32 scratch, row stride LDT
@@ -709,7 +739,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
       for (int i = 0; i < 16; ++i) tinv[(16 * b + i) * LDN + 16 * b + c] = x[i];
     }
-    __syncthreads();
+    named_bar_sync(kTinvBar, kTinvThreads);
     // (b) the two 16x16 blocks T^{-1}[16p+16][16p] (p = 0, 2): warp w < 4 owns
     //     pair w >> 1 and 8 output columns (w & 1)
     if (warp < 4) {
@@ -724,31 +754,49 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       e[0] = -e[0]; e[1] = -e[1]; e[2] = -e[2]; e[3] = -e[3];
       store_frag(tinv + R0 * LDN + C0 + n0, LDN, e, lane);
     }
-    __syncthreads();
+    named_bar_sync(kTinvBar, kTinvThreads);
     // (c) the lower-left 32x32 block: warp w < 8 owns rows 16 (w >> 2) .. +16 and
     //     columns 8 (w & 3) .. +8; zero blocks of the triangular factors are skipped
-    if (warp < 8) {
+    {
       const int m0 = 16 * (warp >> 2), n0 = 8 * (warp & 3);
       float d[4] = {0.f, 0.f, 0.f, 0.f};
       // tmp = N[32..63][0..31] T^{-1}[0..31][0..31]: rows k < n0 of the right factor are 0
       warp_mma_tf32_range(d, nae + (32 + m0) * LDN, LDN, tinv, LDN, n0, n0 & ~7, 32, lane);
       store_frag(tmp + m0 * LDT + n0, LDT, d, lane);
-      named_bar_sync(1, 256);
+      named_bar_sync(kTinvBar, kTinvThreads);
       float e[4] = {0.f, 0.f, 0.f, 0.f};
       // T^{-1}[32..63][32..63] tmp: columns k >= m0 + 16 of the left factor are 0
       warp_mma_tf32_range(e, tinv + (32 + m0) * LDN + 32, LDN, tmp, LDT, n0, 0, m0 + 16, lane);
       e[0] = -e[0]; e[1] = -e[1]; e[2] = -e[2]; e[3] = -e[3];
       store_frag(tinv + (32 + m0) * LDN + n0, LDN, e, lane);
     }
-    __syncthreads();
-    // bf16 copy, K-major [i][j]; blocks above the diagonal are zero
-    for (int item = tid; item < 64 * 8; item += kPrepThreads) {
-      const int i = item >> 3, j = (item & 7) * 8;
-      float x[8];
+    named_bar_sync(kTinvBar, kTinvThreads);
+    // bf16 copy, K-major [i][j]; blocks above the diagonal are zero.  Thread
+    // (i, j8): row i, columns 8 j8 .. +7 (rows are 16-byte aligned: LDN = 68)
+    for (int item = tid; item < 64 * 8; item += kTinvThreads) {
+      const int i = item & 63, j = (item >> 6) * 8;
       const bool upper = (j >> 4) > (i >> 4);
+      const float4 *src = reinterpret_cast<const float4 *>(tinv + i * LDN + j);
+      const float4 x0 = upper ? make_float4(0.f, 0.f, 0.f, 0.f) : src[0];
+      const float4 x1 = upper ? make_float4(0.f, 0.f, 0.f, 0.f) : src[1];
+      st16(sX + X_TINVB + kmajor_off(i, j),
+           make_uint4(pack_bf16x2(x0.x, x0.y), pack_bf16x2(x0.z, x0.w), pack_bf16x2(x1.x, x1.y),
+                      pack_bf16x2(x1.z, x1.w)));
+    }
+  } else {
+    // warps 8-15, meanwhile: Y (lanes n, cols i) -> K-major [n][t]
+    mbar_wait(bar_yo, it & 1, hdr, KDA_DEVICE_TIMEOUT);
+    tc_fence_after();
+    const int cg = (warp >> 2) - 2;  // column group: 32 cg .. +31
+    float v[32];
+    tmem_ld32(taddr(tm, 32 * quad, TM_Y + 32 * cg), v);
+    tmem_ld_wait();
 #pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = upper ? 0.f : tinv[i * LDN + j + u];
-      st16(sX + X_TINVB + kmajor_off(i, j), pack8(x));
+    for (int seg = 0; seg < 4; ++seg) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = v[8 * seg + u];
+      st16(sX + X_Y + kmajor_off(lane_row, 32 * cg + 8 * seg), pack8(x));
     }
   }
   fence_async_smem();
@@ -756,31 +804,30 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
   tc_fence_after();
 
-  // ---- 7. W^T = (K e^{Gp})^T T^{-T};  Y^T = V^T (A_w beta)^T ----
+  // ---- 8. W^T = (K e^{Gp})^T T^{-T};  U^T = Y^T T^{-T} ----
   if (tid == 0) {
-    const uint32_t tinvb = smem_u32(sX + X_TINVB);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_W, desc_mnmajor(smem_u32(sK), 16 * kk, 8192),
-               desc_kmajor(tinvb, 16 * kk, 0), idesc_bf16(128, 64, true, false), kk > 0);
+               desc_kmajor(smem_u32(sX + X_TINVB), 16 * kk, 0), idesc_bf16(128, 64, true, false),
+               kk > 0);
     mma_commit(bar_mma);
   } else if (tid == 32) {
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_Y, desc_mnmajor(smem_u32(sV), 16 * kk, 8192),
-               desc_kmajor(smem_u32(sX + X_AWBW), 16 * kk, 0), idesc_bf16(128, 64, true, false),
+      mma_bf16(tm + TM_U, desc_kmajor(smem_u32(sX + X_Y), 16 * kk, 0),
+               desc_kmajor(smem_u32(sX + X_TINVB), 16 * kk, 0), idesc_bf16(128, 64, false, false),
                kk > 0);
     mma_commit(bar_mma);
   }
   __syncwarp();
   mbar_wait(bar_mma, 1, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
-
-  // readback W (lanes c, cols i) -> K-major [c][t]; Y (lanes n, cols i) -> K-major [n][t]
   {
+    // W (lanes c, cols t) -> K-major [c][t]; U (lanes n, cols t) -> K-major [n][t]
     float v[16], v2[16];
     tmem_ld16(taddr(tm, 32 * quad, TM_W + 16 * qtr), v);
-    tmem_ld16(taddr(tm, 32 * quad, TM_Y + 16 * qtr), v2);
+    tmem_ld16(taddr(tm, 32 * quad, TM_U + 16 * qtr), v2);
     tmem_ld_wait();
 #pragma unroll
     for (int seg = 0; seg < 2; ++seg) {
@@ -791,7 +838,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         y[u] = v2[8 * seg + u];
       }
       st16(sX + X_W + kmajor_off(lane_row, 16 * qtr + 8 * seg), pack8(x));
-      st16(sX + X_Y + kmajor_off(lane_row, 16 * qtr + 8 * seg), pack8(y));
+      st16(sX + X_U + kmajor_off(lane_row, 16 * qtr + 8 * seg), pack8(y));
     }
   }
   fence_async_smem();
@@ -799,66 +846,28 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
   tc_fence_after();
 
-  // ---- 8. U^T = Y^T T^{-T};  K_b^T beta W (for P);  X = W^T (B_e beta)^T (for Q');
-  //         O_intra = tril(B_w) beta V (rows t < 64 of an M = 128 product whose
-  //         upper 64 rows read the bytes after the operand and are discarded) ----
-  if (tid == 0) {
-    const uint32_t tinvb = smem_u32(sX + X_TINVB), wsm = smem_u32(sX + X_W);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_U, desc_kmajor(smem_u32(sX + X_Y), 16 * kk, 0), desc_kmajor(tinvb, 16 * kk, 0),
-               idesc_bf16(128, 64, false, false), kk > 0);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_X, desc_kmajor(wsm, 16 * kk, 0), desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0),
-               idesc_bf16(128, 64, false, false), kk > 0);
-    mma_commit(bar_mma);
-  } else if (tid == 32) {
+  // ---- 9. thread 32: K_b^T beta W (for P), X = W^T (B_e beta)^T (for Q');
+  //         thread 0: O_intra -= tril(B_e) beta U (M = 128 as in step 6),
+  //         Qc = (beta K e^{G_L-G})^T V - (beta K e^{G_L-Gp})^T U (lanes i, columns j) ----
+  if (tid == 32) {
     const uint32_t wsm = smem_u32(sX + X_W);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_OI, desc_kmajor(smem_u32(sX + X_AWBW + 64 * 128), 16 * kk, 0),
-               desc_mnmajor(smem_u32(sV), 16 * kk, 8192), idesc_bf16(128, 128, false, true),
-               kk > 0);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_P, desc_mnmajor(smem_u32(sm + OFF_KBB), 16 * kk, 8192), desc_kmajor(wsm, 16 * kk, 0),
                idesc_bf16(128, 128, true, false), kk > 0);
-    mma_commit(bar_mma);
-  }
-  __syncwarp();
-  mbar_wait(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);
-  tc_fence_after();
-
-  {
-    // U (lanes n, cols t) -> K-major [n][t], the left operand of the last products
-    float u16[16];
-    tmem_ld16(taddr(tm, 32 * quad, TM_U + 16 * qtr), u16);
-    tmem_ld_wait();
 #pragma unroll
-    for (int seg = 0; seg < 2; ++seg) {
-      float x[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) x[u] = u16[8 * seg + u];
-      st16(sX + X_U + kmajor_off(lane_row, 16 * qtr + 8 * seg), pack8(x));
-    }
-  }
-  fence_async_smem();
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-
-  // ---- 9. O_intra -= tril(B_e) beta U (M = 128 as in step 8);
-  //         Qc = (beta K e^{G_L-G})^T V - (beta K e^{G_L-Gp})^T U: lanes i, columns j ----
-  if (tid == 32) {
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tm + TM_X, desc_kmajor(wsm, 16 * kk, 0), desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0),
+               idesc_bf16(128, 64, false, false), kk > 0);
+    mma_commit(bar_px);
+  } else if (tid == 0) {
     const uint32_t usm = smem_u32(sX + X_U);
+    // the first O_intra term (thread 32) has completed: every thread passed bar_yo's
+    // phase before the W/U round
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_OI, desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0), desc_kmajor(usm, 16 * kk, 0),
                idesc_bf16(128, 128, false, false, true), 1);
-    mma_commit(bar_mma);
-  } else if (tid == 0) {
-    const uint32_t usm = smem_u32(sX + X_U);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sm + OFF_KAB), 16 * kk, 8192),
@@ -868,8 +877,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sm + OFF_KBB), 16 * kk, 8192),
                desc_kmajor(usm, 16 * kk, 0), idesc_bf16(128, 128, true, false, true), 1);
-    mma_commit(bar_mma);
+    mma_commit(bar_oq);
   }
+  __syncwarp();
+  mbar_wait(bar_px, it & 1, hdr, KDA_DEVICE_TIMEOUT);
+  tc_fence_after();
   // P and Q' leave TMEM for the slot while the last products run (disjoint columns)
   {
     float v[32], x16[16];
@@ -904,18 +916,17 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       st16(sX + X_QPI + sw128((uint32_t)(c * 128 + (16 * qtr + 8 * seg) * 2)), pack8(x));
     }
   }
-
   fence_async_smem();
-  __syncwarp();
-  mbar_wait(bar_mma, 1, hdr, KDA_DEVICE_TIMEOUT);
+  tc_fence_before();
+  __syncthreads();  // the P / Q' images are written
   tc_fence_after();
-  __syncthreads();  // the P / Q' images are written and every read of the q tile is done
-
   if (tid == 0) {  // P and Q' images -> workspace slot
     bulk_s2g(slot + SLOT_P, sX + X_PI, 32768);
     bulk_s2g(slot + SLOT_QP, sX + X_QPI, 16384);
     bulk_commit();
   }
+  mbar_wait(bar_oq, it & 1, hdr, KDA_DEVICE_TIMEOUT);
+  tc_fence_after();
   // the input tiles are consumed: start the next item's loads now
   if (tid == 0 && next < total) load_qkv(next, ce_next);
   if (tid < C && next < total) load_beta(next, ce_next, nbeta, ngsc);
