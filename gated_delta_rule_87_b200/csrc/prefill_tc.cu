@@ -564,53 +564,56 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       w0[r] = w0[r + 1] * a0[r + 1];
       w1[r] = w1[r + 1] * a1[r + 1];
     }
-    float pq0 = pre0, pq1 = pre1;  // prefix product through t-1: e^{Gp_t - E_{I-1}}
+    // Channel pairs in packed fp32x2 arithmetic.  Every operand row written
+    // here has the same residue mod 8 as t, so the SW128 position of channel
+    // pair c2 within a 128-byte row is one offset per row.
+    const float2 fa = make_float2(fa0, fa1), fb = make_float2(fb0, fb1), rf = make_float2(rf0, rf1);
+    const float2 ei = make_float2(ei0, ei1), ge = make_float2(ge0, ge1);
+    const uint32_t cblk = (uint32_t)(c2 >> 6), cpos = (uint32_t)(c2 & 63) * 2;  // byte in the row
+    unsigned char *const rbase = sX + X_R + cblk * 16384;
+    unsigned char *const lbase = sX + X_LEFT + cblk * LEFT_BLOCK;
+    unsigned char *const kbase = sK + cblk * 8192, *const qbase = sQ + cblk * 8192;
+    unsigned char *const abase = sm + OFF_KAB + cblk * 8192, *const bbase = sm + OFF_KBB + cblk * 8192;
+    auto st4 = [](unsigned char *p, float2 x) {
+      *reinterpret_cast<uint32_t *>(p) = pack_bf16x2(x.x, x.y);
+    };
+    float2 pq = make_float2(pre0, pre1);  // prefix product through t-1: e^{Gp_t - E_{I-1}}
 #pragma unroll
     for (int r = 0; r < 8; ++r) {
       const int t = 16 * bI + 8 * rh + r;
-      const uint32_t koff = (c2 >> 6) * 8192 + kmajor_off(t, c2 & 63);
-      const uint32_t kraw = *reinterpret_cast<const uint32_t *>(sK + koff);
-      const uint32_t qraw = *reinterpret_cast<const uint32_t *>(sQ + koff);
+      const uint32_t x = (cpos ^ ((uint32_t)(t & 7) << 4));  // swizzled byte within a row
+      const uint32_t koff = (uint32_t)t * 128 + x;
+      const uint32_t kraw = *reinterpret_cast<const uint32_t *>(kbase + koff);
+      const uint32_t qraw = *reinterpret_cast<const uint32_t *>(qbase + koff);
       const bool ok = t < L;
-      const float k0 = ok ? bf16_lo(kraw) : 0.f, k1 = ok ? bf16_hi(kraw) : 0.f;
-      const float q0 = ok ? bf16_lo(qraw) : 0.f, q1 = ok ? bf16_hi(qraw) : 0.f;
+      const float2 k = ok ? make_float2(bf16_lo(kraw), bf16_hi(kraw)) : make_float2(0.f, 0.f);
+      const float2 q = ok ? make_float2(bf16_lo(qraw), bf16_hi(qraw)) : make_float2(0.f, 0.f);
       const float b = sBeta[t];
-      const float bq0 = pq0 * a0[r], bq1 = pq1 * a1[r];       // e^{G_t - E_{I-1}}
-      const float bk0 = DECAY_FIRST ? bq0 : pq0;              // e^{Gp_t - E_{I-1}}
-      const float bk1 = DECAY_FIRST ? bq1 : pq1;
-      const float rw0 = w0[r], rw1 = w1[r];                   // e^{E_I - G_t}
-      const float re0 = DECAY_FIRST ? rw0 : rw0 * a0[r];      // e^{E_I - Gp_t}
-      const float re1 = DECAY_FIRST ? rw1 : rw1 * a1[r];
-      pq0 = bq0;
-      pq1 = bq1;
-      const int rowK = 32 * bI + 8 * rh + r, rowQ = rowK + 16;
+      const float2 a = make_float2(a0[r], a1[r]);
+      const float2 bq = __fmul2_rn(pq, a);                    // e^{G_t - E_{I-1}}
+      const float2 bk = DECAY_FIRST ? bq : pq;                // e^{Gp_t - E_{I-1}}
+      const float2 rw = make_float2(w0[r], w1[r]);            // e^{E_I - G_t}
+      const float2 re = DECAY_FIRST ? rw : __fmul2_rn(rw, a); // e^{E_I - Gp_t}
+      pq = bq;
+      const float2 kw = __fmul2_rn(k, rw), ke = __fmul2_rn(k, re);
+      const float2 kb = __fmul2_rn(k, bk), qb = __fmul2_rn(q, bq);
+      const uint32_t rowK = (uint32_t)(32 * bI + 8 * rh + r) * 128 + x, rowQ = rowK + 16 * 128;
       // Gram right operand (keys scaled to their group's anchor)
-      const uint32_t rb = X_R + (c2 >> 6) * 16384;
-      *reinterpret_cast<uint32_t *>(sX + rb + kmajor_off(rowK, c2 & 63)) =
-          pack_bf16x2(k0 * rw0 * rf0, k1 * rw1 * rf1);
-      *reinterpret_cast<uint32_t *>(sX + rb + kmajor_off(rowQ, c2 & 63)) =
-          pack_bf16x2(k0 * re0 * rf0, k1 * re1 * rf1);
+      st4(rbase + rowK, __fmul2_rn(kw, rf));
+      st4(rbase + rowQ, __fmul2_rn(ke, rf));
       // Gram left operands: anchor E_0 (all rows), anchor E_2 (sub-chunks 2, 3)
-      {
-        const uint32_t lb = X_LEFT + (c2 >> 6) * LEFT_BLOCK;
-        *reinterpret_cast<uint32_t *>(sX + lb + kmajor_off(rowK, c2 & 63)) =
-            pack_bf16x2(k0 * bk0 * fa0, k1 * bk1 * fa1);
-        *reinterpret_cast<uint32_t *>(sX + lb + kmajor_off(rowQ, c2 & 63)) =
-            pack_bf16x2(q0 * bq0 * fa0, q1 * bq1 * fa1);
-        if (bI >= 2) {
-          *reinterpret_cast<uint32_t *>(sX + lb + LEFT_G1 + kmajor_off(rowK, c2 & 63)) =
-              pack_bf16x2(k0 * bk0 * fb0, k1 * bk1 * fb1);
-          *reinterpret_cast<uint32_t *>(sX + lb + LEFT_G1 + kmajor_off(rowQ, c2 & 63)) =
-              pack_bf16x2(q0 * bq0 * fb0, q1 * bq1 * fb1);
-        }
+      st4(lbase + rowK, __fmul2_rn(kb, fa));
+      st4(lbase + rowQ, __fmul2_rn(qb, fa));
+      if (bI >= 2) {
+        st4(lbase + LEFT_G1 + rowK, __fmul2_rn(kb, fb));
+        st4(lbase + LEFT_G1 + rowQ, __fmul2_rn(qb, fb));
       }
       // K e^{Gp} over k, q e^{G} over q (same element, same owner), beta K e^{G_L - G|Gp}
-      *reinterpret_cast<uint32_t *>(sK + koff) = pack_bf16x2(k0 * bk0 * ei0, k1 * bk1 * ei1);
-      *reinterpret_cast<uint32_t *>(sQ + koff) = pack_bf16x2(q0 * bq0 * ei0, q1 * bq1 * ei1);
-      *reinterpret_cast<uint32_t *>(sm + OFF_KAB + koff) =
-          pack_bf16x2(b * k0 * rw0 * ge0, b * k1 * rw1 * ge1);
-      *reinterpret_cast<uint32_t *>(sm + OFF_KBB + koff) =
-          pack_bf16x2(b * k0 * re0 * ge0, b * k1 * re1 * ge1);
+      st4(kbase + koff, __fmul2_rn(kb, ei));
+      st4(qbase + koff, __fmul2_rn(qb, ei));
+      const float2 bge = __fmul2_rn(make_float2(b, b), ge);
+      st4(abase + koff, __fmul2_rn(kw, bge));
+      st4(bbase + koff, __fmul2_rn(ke, bge));
     }
   }
   fence_async_smem();
@@ -640,45 +643,58 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   const int lane_row = 32 * quad + lane;
 
   // ---- 5. Gram readback: masked, beta-scaled, into the next operands ----
+  // Warp (I = quad, J = qtr) holds rows of query/key sub-chunk I against keys of
+  // sub-chunk J.  Blocks with J > I are zero; inside J == I the strict (keys) or
+  // inclusive (queries) lower triangle survives.  Rows and keys past the chunk's
+  // length are zero already (k = q = beta = 0 there).
   {
-    const int I = quad, s = lane;
+    const int I = quad, J = qtr, s = lane;
     const bool isK = s < 16;
     const int i = 16 * I + (s & 15);
     float* nae = reinterpret_cast<float *>(sX + X_NAE);
-    {
-      const int J = qtr;
+    float w[16], e[16];
+    if (J <= I) {  // warp-uniform
       float v[32];
       tmem_ld32(taddr(tm, 32 * quad, TM_GRAM + 32 * J), v);
+      float bj[16];
+#pragma unroll
+      for (int u = 0; u < 16; u += 4) {
+        const float4 b4 = *reinterpret_cast<const float4 *>(sBeta + 16 * J + u);
+        bj[u] = b4.x; bj[u + 1] = b4.y; bj[u + 2] = b4.z; bj[u + 3] = b4.w;
+      }
       tmem_ld_wait();
-      float w[16], e[16];
+      const int lim = J < I ? 16 : (isK ? (s & 15) : (s & 15) + 1);  // keys u < lim survive
 #pragma unroll
       for (int u = 0; u < 16; ++u) {
-        const int j = 16 * J + u;
-        const bool ok = (J <= I) && (i < L) && (j < L) && (isK ? (j < i) : (j <= i));
-        w[u] = ok ? v[u] * sBeta[j] : 0.f;
-        e[u] = ok ? v[16 + u] * sBeta[j] : 0.f;
+        w[u] = u < lim ? v[u] * bj[u] : 0.f;
+        e[u] = u < lim ? v[16 + u] * bj[u] : 0.f;
       }
-      const int row_w = isK ? i : 64 + i;
+    } else {
 #pragma unroll
-      for (int hseg = 0; hseg < 2; ++hseg) {
-        float x[8];
+      for (int u = 0; u < 16; ++u) w[u] = e[u] = 0.f;
+    }
+    const int row_w = isK ? i : 64 + i;
 #pragma unroll
-        for (int u = 0; u < 8; ++u) x[u] = w[8 * hseg + u];
-        st16(sX + X_AWBW + kmajor_off(row_w, 16 * J + 8 * hseg), pack8(x));
-      }
-      if (isK) {
+    for (int hseg = 0; hseg < 2; ++hseg) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = w[8 * hseg + u];
+      st16(sX + X_AWBW + kmajor_off(row_w, 16 * J + 8 * hseg), pack8(x));
+    }
+    if (isK) {
+      if (J <= I) {  // T^{-1} reads N only on and below the diagonal blocks
 #pragma unroll
         for (int u = 0; u < 16; u += 4)
           *reinterpret_cast<float4 *>(nae + i * LDN + 16 * J + u) =
               make_float4(e[u], e[u + 1], e[u + 2], e[u + 3]);
-      } else {
+      }
+    } else {
 #pragma unroll
-        for (int hseg = 0; hseg < 2; ++hseg) {
-          float x[8];
+      for (int hseg = 0; hseg < 2; ++hseg) {
+        float x[8];
 #pragma unroll
-          for (int u = 0; u < 8; ++u) x[u] = e[8 * hseg + u];
-          st16(sX + X_BE + kmajor_off(i, 16 * J + 8 * hseg), pack8(x));
-        }
+        for (int u = 0; u < 8; ++u) x[u] = e[8 * hseg + u];
+        st16(sX + X_BE + kmajor_off(i, 16 * J + 8 * hseg), pack8(x));
       }
     }
   }
