@@ -214,6 +214,7 @@ plan_kernel(const int32_t *__restrict__ cu, int num_seqs, int T, int T_total, in
 // prep kernel
 // ---------------------------------------------------------------------------
 constexpr int kPrepThreads = 512;
+constexpr int kIoThread = 480;  // issues the TMA loads and image stores (lane 0 of the last warp)
 
 // shared memory map (bytes from a 1024-aligned base)
 constexpr uint32_t OFF_Q = 0;         // q tile, two K-major SW128 [64 t][64 c] blocks; later q.e^{G}
@@ -434,7 +435,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   };
   float nbeta = 0.f, ngsc = 0.f;  // the coming item's, loaded one item ahead
   ChunkEntry ce = entry(work), ce_next = entry(work + gridDim.x);
-  if (tid == 0) {
+  if (tid == kIoThread) {
     load_g(work, ce);
     load_qkv(work, ce);
     if (work + (int)gridDim.x < total) prefetch_l2(work + gridDim.x, ce_next);
@@ -511,9 +512,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   }
   // the previous item's image copies must have read the X region before it is rebuilt
-  if (tid == 0) bulk_wait_read0();
+  if (tid == kIoThread) bulk_wait_read0();
   __syncthreads();  // g is consumed: the next item's lands there
-  if (tid == 0 && next < total) {
+  if (tid == kIoThread && next < total) {
     load_g(next, ce_next);
     if (next + (int)gridDim.x < total) prefetch_l2(next + gridDim.x, ce_next2);
   }
@@ -704,14 +705,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   //         Y^T = V^T (A_w beta)^T;  O_intra = tril(B_w) beta V (rows t < 64 of an
   //         M = 128 product whose upper 64 rows read the bytes after the operand
   //         and are discarded) ----
-  if (tid == 0) {
+  if (tid == 256) {
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_Y, desc_mnmajor(smem_u32(sV), 16 * kk, 8192),
                desc_kmajor(smem_u32(sX + X_AWBW), 16 * kk, 0), idesc_bf16(128, 64, true, false),
                kk > 0);
     mma_commit(bar_yo);
-  } else if (tid == 32) {
+  } else if (tid == 288) {
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_OI, desc_kmajor(smem_u32(sX + X_AWBW + 64 * 128), 16 * kk, 0),
@@ -878,8 +879,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mma_commit(bar_px);
   } else if (tid == 0) {
     const uint32_t usm = smem_u32(sX + X_U);
-    // the first O_intra term (thread 32) has completed: every thread passed bar_yo's
-    // phase before the W/U round
+    // the first O_intra term (thread 288) has completed: warps 8-15 passed bar_yo's
+    // phase before the barrier ahead of the W/U round
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_OI, desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0), desc_kmajor(usm, 16 * kk, 0),
@@ -936,7 +937,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   tc_fence_before();
   __syncthreads();  // the P / Q' images are written
   tc_fence_after();
-  if (tid == 0) {  // P and Q' images -> workspace slot
+  if (tid == kIoThread) {  // P and Q' images -> workspace slot
     bulk_s2g(slot + SLOT_P, sX + X_PI, 32768);
     bulk_s2g(slot + SLOT_QP, sX + X_QPI, 16384);
     bulk_commit();
@@ -944,7 +945,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   mbar_wait(bar_oq, it & 1, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
   // the input tiles are consumed: start the next item's loads now
-  if (tid == 0 && next < total) load_qkv(next, ce_next);
+  if (tid == kIoThread && next < total) load_qkv(next, ce_next);
   if (tid < C && next < total) load_beta(next, ce_next, nbeta, ngsc);
   {
     // warp (quad, qtr) holds rows 32 quad + lane, value columns 32 qtr .. +31,
@@ -975,7 +976,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid == 0) {  // Qc and O_intra images -> workspace slot
+  if (tid == kIoThread) {  // Qc and O_intra images -> workspace slot
     bulk_s2g(slot + SLOT_QC, sX + X_QCI, 32768);
     bulk_s2g(slot + SLOT_OI, sX + X_OII, 16384);
     bulk_commit();
@@ -984,7 +985,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   ce_next = ce_next2;
   }  // work items
 
-  if (tid == 0) bulk_wait0();
+  if (tid == kIoThread) bulk_wait0();
   tc_fence_before();
   __syncthreads();
   if (warp == 0) tmem_dealloc(tm, 512);
