@@ -426,7 +426,8 @@ def bench_decode(args, device, world, peaks, stream, flush):
             "value": round(gbs * world, 1), "unit": "GB/s (state read+write and token I/O)",
             "roofline": {"bound": "hbm", "achieved": round(gbs, 1), "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": round(gbs / peaks["hbm_gbs"], 4),
-                         "traffic": None, "peak_source": peaks["source"],
+                         "traffic": measured_traffic("recurrent_kernel", w.name),
+                         "peak_source": peaks["source"],
                          "kernel": "recurrent_kernel"},
             "l2": "state (512 MB) larger than L2; not flushed",
             "launches": w.steps}
