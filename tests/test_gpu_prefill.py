@@ -161,3 +161,18 @@ def test_kda_varlen_full_workload_sampled_heads():
 def test_gdn_long_full_workload_sampled_heads():
     x = W.make_prefill(W.WORKLOADS["gdn_long"], seed=0)
     _check(x, heads=[0, 1, 30])
+
+
+@pytest.mark.parametrize("nseq", [8, 20])
+def test_kda_column_slice_widths(nseq):
+    """The scan splits each (sequence, v-head) state into 32-column slices (4
+    CTAs) while the chains fit on the SMs in one wave, else 64-column slices
+    (2 CTAs): both widths must agree with the oracle.  With 2 heads, 8
+    sequences give 64 four-way chains (narrow); 20 give 160 > 148 SMs (wide)."""
+    import torch
+    sms = torch.cuda.get_device_properties(0).multi_processor_count
+    assert (nseq * 2 * 4 <= sms) == (nseq == 8)
+    w = W.WORKLOADS["kda_varlen"].replace(H_qk=2, H_v=2, init_state=True)
+    rng = np.random.default_rng(12 + nseq)
+    lengths = [int(x) for x in rng.integers(1, 200, nseq)]
+    _check(W.make_prefill(w, seed=12, lengths=lengths))
