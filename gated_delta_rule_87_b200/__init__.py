@@ -34,6 +34,8 @@ library_path = os.path.join(_PKG, "libgated_delta.so")
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_DEVICE_CHECK, \
     KDA_ERR_WORKSPACE = range(6)
 KDA_F32, KDA_BF16 = 0, 1
+# device codes in a workspace's status word (kda_check_device_status)
+KDA_DEVICE_OK, KDA_DEVICE_BAD_CU_SEQLENS, KDA_DEVICE_TIMEOUT = 0, 1, 2
 # decay order (KDA): the table's literal order, or the decay applied before the erase
 ERASE_THEN_DECAY, DECAY_THEN_ERASE = "erase_then_decay", "decay_then_erase"
 _ORDER = {ERASE_THEN_DECAY: 0, DECAY_THEN_ERASE: 1}
@@ -44,7 +46,7 @@ EXPORTED_SYMBOLS = (
     "kda_check_device_status", "kda_status_string", "kda_last_error", "kda_abi_version",
     "kda_trace_enable", "kda_trace_read", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_ex",
     "gdn_chunk_fwd_ex", "kda_recurrent_fwd", "gdn_recurrent_fwd", "kda_state_gather",
-    "kda_state_scatter",
+    "kda_state_scatter", "kda_selftest_wait_timeout",
 )
 
 _lock = threading.Lock()
@@ -66,6 +68,7 @@ _SIGS = {
     "kda_decode_step": ([_vp] * 7 + [_i32] * 4 + [ctypes.c_int, _vp], ctypes.c_int),
     "gdn_decode_step": ([_vp] * 7 + [_i32] * 5 + [ctypes.c_int, _vp], ctypes.c_int),
     "kda_check_device_status": ([_vp, _vp, ctypes.POINTER(_i32)], ctypes.c_int),
+    "kda_selftest_wait_timeout": ([_vp, _i32, _vp], ctypes.c_int),
     "kda_status_string": ([ctypes.c_int], ctypes.c_char_p),
     "kda_last_error": ([], ctypes.c_char_p),
     "kda_abi_version": ([], _i32),
@@ -367,6 +370,17 @@ def trace_read(capacity: int = 4096):
     n = L.kda_trace_read(names, stride, ms, capacity)
     return [(names.raw[i * stride:(i + 1) * stride].split(b"\0", 1)[0].decode(), float(ms[i]))
             for i in range(n)]
+
+
+def selftest_wait_timeout(workspace, max_polls: int = 16, stream=None) -> None:
+    """Run one bounded on-device wait that nothing completes; it expires and
+    writes KDA_DEVICE_TIMEOUT into ``workspace``'s status word (read it with
+    check_device_status).  Exercises the library's expired-wait path without
+    faulting or hanging the GPU."""
+    L = lib()
+    _check(L.kda_selftest_wait_timeout(_ptr(workspace), int(max_polls),
+                                       _stream_handle(stream, workspace.device)),
+           "kda_selftest_wait_timeout")
 
 
 def check_device_status(workspace, stream=None) -> Tuple[int, int]:

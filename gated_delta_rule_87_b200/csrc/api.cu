@@ -359,6 +359,19 @@ kda_status_t kda_state_scatter(const float *src, float *pool, const int32_t *sta
   return state_copy_common(src, nullptr, N, pool, state_slots, num_slots, N, H, d_k, d_v, stream);
 }
 
+kda_status_t kda_selftest_wait_timeout(void *workspace, int32_t max_polls, void *stream) {
+  if (!workspace) return fail(KDA_ERR_INVALID_ARG, "workspace is NULL");
+  if (max_polls < 1 || max_polls > 4096)
+    return fail(KDA_ERR_INVALID_ARG, "max_polls must be in [1, 4096]");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t *status = static_cast<int32_t *>(workspace);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
+  e = gdr::launch_wait_timeout(status, (uint32_t)max_polls, s);
+  if (e != cudaSuccess) return cuda_fail(e, "wait-timeout launch");
+  return KDA_OK;
+}
+
 kda_status_t kda_check_device_status(const void *workspace, void *stream, int32_t *device_code) {
   if (!workspace) return fail(KDA_ERR_INVALID_ARG, "workspace is NULL");
   int32_t code = 0;

@@ -54,6 +54,9 @@ cudaError_t launch_state_copy(const float *src, const int32_t *src_slots, int64_
                               float *dst, const int32_t *dst_slots, int64_t dst_limit, int N,
                               int64_t per_seq_floats, cudaStream_t stream);
 
+// One bounded on-device wait that expires: writes KDA_DEVICE_TIMEOUT to *status.
+cudaError_t launch_wait_timeout(int32_t *status, uint32_t max_polls, cudaStream_t stream);
+
 // Chunk length of the prefill kernels (tokens per chunk).
 constexpr int kChunk = 64;
 

@@ -92,9 +92,9 @@ constexpr uint32_t kMaxPolls = 4096;
 // raises *err, when given) if the bound is hit; the caller then skips its
 // remaining work instead of hanging.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_t *err,
-                                          int32_t code) {
+                                          int32_t code, uint32_t max_polls = kMaxPolls) {
   if (mbar_test_wait(bar, parity)) return true;
-  for (uint32_t i = 0; i < kMaxPolls; ++i)
+  for (uint32_t i = 0; i < max_polls; ++i)
     if (mbar_try_wait(bar, parity)) return true;
   if (err) atomicExch(err, code);
   return false;

@@ -292,6 +292,18 @@ KDA_API kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, const v
 KDA_API kda_status_t kda_check_device_status(const void *workspace, void *stream,
                                      int32_t *device_code);
 
+/* Diagnostic: runs one on-device wait that nothing ever completes, bounded like
+ * every wait in the library's kernels (an mbarrier poll loop of at most
+ * max_polls polls, each at most ~1 ms).  When the bound expires the kernel
+ * writes KDA_DEVICE_TIMEOUT into the status word at the start of `workspace`
+ * (any prefill workspace, or 4 bytes of device memory) and returns, exactly as
+ * an expired wait inside a prefill does; kda_check_device_status() then
+ * reports it.  Lets a caller test its handling of an expired wait without
+ * faulting or hanging the GPU.  The status word is reset to KDA_DEVICE_OK
+ * first.  max_polls in [1, 4096]; returns KDA_ERR_INVALID_ARG otherwise (or
+ * for a NULL workspace) before touching the device.  Asynchronous on `stream`. */
+KDA_API kda_status_t kda_selftest_wait_timeout(void *workspace, int32_t max_polls, void *stream);
+
 /* Static text for a status code. */
 KDA_API const char *kda_status_string(kda_status_t status);
 

@@ -171,3 +171,12 @@ def test_state_scatter_validation():
     assert L.kda_state_scatter(FAKE, FAKE + 4096, None, 8, 4, 2, 128, 128, None) == \
         gdr.KDA_ERR_INVALID_ARG
     assert L.kda_state_scatter(None, None, None, 0, 0, 2, 128, 128, None) == gdr.KDA_OK
+
+
+def test_selftest_wait_timeout_validates_on_host():
+    """Argument checks run before the device is touched (no GPU needed)."""
+    L = gdr.lib()
+    assert L.kda_selftest_wait_timeout(None, 16, None) == gdr.KDA_ERR_INVALID_ARG
+    dummy = ctypes.c_void_p(256)  # never dereferenced: the bound check fails first
+    assert L.kda_selftest_wait_timeout(dummy, 0, None) == gdr.KDA_ERR_INVALID_ARG
+    assert L.kda_selftest_wait_timeout(dummy, 5000, None) == gdr.KDA_ERR_INVALID_ARG
