@@ -134,8 +134,9 @@ plan_kernel(const int32_t *__restrict__ cu, int num_seqs, int T, int T_total, in
       if (i < num_seqs && cu[i + 1] < x) bad = true;
     }
   }
-  if (__syncthreads_or(bad)) {
+  if (__syncthreads_or(bad)) {  // every table entry stays in bounds
     for (int i = tid; i <= num_seqs; i += blockDim.x) seq_off[i] = 0;
+    for (int i = tid; i < num_seqs; i += blockDim.x) order[i] = i;
     if (tid == 0) {
       hdr[0] = KDA_DEVICE_BAD_CU_SEQLENS;
       hdr[1] = 0;
