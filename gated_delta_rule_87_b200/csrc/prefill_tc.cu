@@ -349,7 +349,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // 1024-byte aligned base, derived by pointer arithmetic on the shared array so
   // that the compiler keeps shared-memory addressing for every access
   unsigned char *sm = smem_raw + ((1024u - (smem_u32(smem_raw) & 1023u)) & 1023u);
-  unsigned char *sQ = sm + OFF_Q, *sK = sm + OFF_K, *sV = sm + OFF_V;
+  // q and k tiles: two K-major SW128 blocks of 64 channels each.  Per-channel
+  // gate: the q blocks, then the k blocks.  Scalar gate: each 16 KB block holds
+  // 64 k rows then 64 q rows, so that [K; Q] is one 128-row MMA operand.
+  constexpr uint32_t QK_CB = CHANNEL ? 8192 : 16384;  // bytes between 64-channel blocks
+  unsigned char *sQ = sm + (CHANNEL ? OFF_Q : OFF_Q + 8192), *sK = sm + (CHANNEL ? OFF_K : OFF_Q);
+  unsigned char *sV = sm + OFF_V;
+  // k e^{Gp} and q e^{G} as the later products read them (64-channel blocks
+  // 8 KB apart): in place per-channel, in the g buffer with a scalar gate
+  unsigned char *sKd = CHANNEL ? sK : sm + OFF_G, *sQd = CHANNEL ? sQ : sm + OFF_G + 16384;
   float *sG = reinterpret_cast<float *>(sm + OFF_G);
   unsigned char *sX = sm + OFF_X;
   float *sBeta = reinterpret_cast<float *>(sm + OFF_MISC + MISC_BETA);
@@ -411,8 +419,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mbar_arrive_expect_tx(bar_tma, 3 * 16384);
 #pragma unroll
     for (int cb = 0; cb < 2; ++cb) {
-      tma_load_3d(sQ + cb * 8192, &tm_q, cb * 64, hkk, ts, bar_tma);
-      tma_load_3d(sK + cb * 8192, &tm_k, cb * 64, hkk, ts, bar_tma);
+      tma_load_3d(sQ + cb * QK_CB, &tm_q, cb * 64, hkk, ts, bar_tma);
+      tma_load_3d(sK + cb * QK_CB, &tm_k, cb * 64, hkk, ts, bar_tma);
       tma_load_3d(sV + cb * 8192, &tm_v, cb * 64, hh, ts, bar_tma);
     }
   };
@@ -456,7 +464,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   mbar_wait(bar_tma, it & 1, hdr, KDA_DEVICE_TIMEOUT);
   __syncthreads();
+  // readbacks: warp (quad, qtr) reads TMEM lanes 32*quad .. +31, column quarter qtr
+  const int quad = warp & 3, qtr = warp >> 2;
+  const int lane_row = 32 * quad + lane;
 
+  if constexpr (CHANNEL) {
   // ---- 2. per-token decays a = e^{g} (rows >= L: no decay), sub-chunk sums ----
   // Thread (I, h, p) owns channels c = 2p, 2p+1 of tokens 8h .. 8h+7 of
   // sub-chunk I; a warp spans 64 channels of the same rows, so its 4-byte
@@ -640,10 +652,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   mbar_wait(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
 
-  // readbacks: warp (quad, qtr) reads TMEM lanes 32*quad .. +31, column quarter qtr
-  const int quad = warp & 3, qtr = warp >> 2;
-  const int lane_row = 32 * quad + lane;
-
   // ---- 5. Gram readback: masked, beta-scaled, into the next operands ----
   // Warp (I = quad, J = qtr) holds rows of query/key sub-chunk I against keys of
   // sub-chunk J.  Blocks with J > I are zero; inside J == I the strict (keys) or
@@ -700,7 +708,215 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
     }
   }
+  fence_async_smem();  // the images are operands of the next products
   __syncthreads();
+  } else {
+  // ---- 2'. scalar gate: every decay factor is a per-token scalar, so the Gram
+  //          products take the raw tiles and the factors are applied to the
+  //          64 x 64 results.  [K; Q] K^T is issued as soon as the tiles land ----
+  if (tid == 0) {
+    tc_fence_after();
+    constexpr uint32_t ID = idesc_bf16(128, 64, false, false);
+    const uint32_t kq = smem_u32(sK);  // rows 0..63: k, rows 64..127: q
+#pragma unroll
+    for (int kk = 0; kk < 8; ++kk)
+      mma_bf16(tm + TM_GRAM, desc_kmajor(kq, 16 * kk, QK_CB), desc_kmajor(kq, 16 * kk, QK_CB), ID,
+               kk > 0);
+    mma_commit(bar_mma);
+    mma_commit(bar_mma);  // the phase counts two commits
+  }
+  // Per-token tables, warp 1 (lane: tokens 2 lane, 2 lane + 1).  G_t is the
+  // in-chunk cumulative log-decay through t, Gp_t through t - 1, E_J its value
+  // at the end of 16-token block J, G_L at the end of the chunk (g = 0 past
+  // the chunk's length).  Every factor is e^{x} with x <= 0:
+  //   a_t = e^{g_t}; e^{Gp_t} (K for W); e^{G_t} (q for Q');
+  //   beta_t e^{G_L - G_t}, beta_t e^{G_L - Gp_t} (K_a, K_b);
+  //   beta_t e^{E_J - G_t} (key column factor of the Gram blocks left of the diagonal).
+  // Rows past the chunk's length get 0 in the tile factors.
+  float *tG = sPblk, *tGp = sPblk + 64, *tA = sPblk + 128, *tCW = sPblk + 192, *tE = sPblk + 256;
+  float *tFK = sGsum, *tFQ = sGsum + 64, *tFA = sGsum + 128, *tFB = sGsum + 192;
+  // diagonal-block factors [4 blocks][16 rows][kLdD] (the per-channel path's
+  // half-sub-chunk scratch; no image copy reads it)
+  constexpr int kLdD = 20;  // padded row: two-way bank conflicts at most
+  float *tD = reinterpret_cast<float *>(sm + OFF_MISC + MISC_XP);
+  if (warp == 1) {
+    const int t0 = 2 * lane, t1 = t0 + 1;
+    const float g0 = sGsc[t0], g1 = sGsc[t1];  // 0 past the chunk's length
+    float incl = g0 + g1;  // inclusive scan of token pairs over the lanes
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const float y = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += y;
+    }
+    float excl = __shfl_up_sync(0xffffffffu, incl, 1);
+    if (lane == 0) excl = 0.f;
+    const float G0 = excl + g0, G1 = G0 + g1;
+    const float GL = __shfl_sync(0xffffffffu, G1, 31);
+    const float EJ = __shfl_sync(0xffffffffu, G1, lane | 7);  // end of this lane's 16-token block
+    const float gle = expf(GL);
+#pragma unroll
+    for (int h2 = 0; h2 < 2; ++h2) {
+      const int t = t0 + h2;
+      const float Gt = h2 ? G1 : G0, Gpt = h2 ? G0 : excl, at = expf(h2 ? g1 : g0);
+      const bool ok = t < L;
+      const float b = sBeta[t];  // 0 past the chunk's length
+      const float fa = b * expf(GL - Gt);
+      tG[t] = Gt;
+      tGp[t] = Gpt;
+      tA[t] = at;
+      tCW[t] = b * expf(EJ - Gt);
+      tFK[t] = ok ? expf(Gpt) : 0.f;
+      tFQ[t] = ok ? expf(Gt) : 0.f;
+      tFA[t] = fa;
+      tFB[t] = fa * at;  // e^{G_L - Gp_t} = e^{G_L - G_t} e^{g_t}
+      sGLe[t] = gle;
+      sGLe[t + C] = gle;
+    }
+    if ((lane & 7) == 7) tE[lane >> 3] = G1;
+  } else if (warp == 2 || warp == 3) {
+    // Diagonal Gram blocks, row a of 16-token block I (thread 16 I + a; a
+    // half-warp per block): D[I][a][b] = e^{Gp_{16I+a} - G_{16I+b}}, the product
+    // of the decays a_s of tokens b < s < a (1 for b = a - 1, 0 for b >= a).
+    // Products of factors <= 1: none overflows.
+    const int I = (tid - 64) >> 4, a = (tid - 64) & 15;
+    const float own = expf(sGsc[16 * I + a]);  // a_{16I+a}
+    float as[16];
+#pragma unroll
+    for (int s2 = 0; s2 < 16; ++s2) as[s2] = __shfl_sync(0xffffffffu, own, (lane & 16) | s2);
+    float d[16], prod = 1.f;
+    d[15] = 0.f;
+#pragma unroll
+    for (int b2 = 14; b2 >= 0; --b2) {
+      prod = (b2 + 1 < a) ? prod * as[b2 + 1] : 1.f;
+      d[b2] = (b2 < a) ? prod : 0.f;
+    }
+    float4 *row = reinterpret_cast<float4 *>(tD + (16 * I + a) * kLdD);
+#pragma unroll
+    for (int q4 = 0; q4 < 4; ++q4) row[q4] = make_float4(d[4 * q4], d[4 * q4 + 1], d[4 * q4 + 2], d[4 * q4 + 3]);
+  }
+  // the previous item's image copies must have read the X region before it is rebuilt
+  if (tid == kIoThread) bulk_wait_read0();
+  __syncthreads();
+  if (tid == kIoThread && next < total) {
+    load_g(next, ce_next);
+    if (next + (int)gridDim.x < total) prefetch_l2(next + gridDim.x, ce_next2);
+  }
+  // ---- 3'. while the Gram runs: the row-scaled tiles the later products read,
+  //          in the per-channel path's layout: k e^{Gp} and q e^{G} (in the g
+  //          buffer, which a scalar gate does not use), beta k e^{G_L - G} and
+  //          beta k e^{G_L - Gp}.  Thread: channel pair c2, rows 8 rg .. +7; a
+  //          warp covers one 128-byte row segment ----
+  {
+    const int c2 = (tid & 63) * 2, rg = tid >> 6;
+    const uint32_t cblk = (uint32_t)(c2 >> 6), cpos = (uint32_t)(c2 & 63) * 2;
+    const unsigned char *const kr = sK + cblk * QK_CB, *const qr = sQ + cblk * QK_CB;
+    unsigned char *const kd = sm + OFF_G + cblk * 8192, *const qd = sm + OFF_G + 16384 + cblk * 8192;
+    unsigned char *const ab = sm + OFF_KAB + cblk * 8192, *const bb = sm + OFF_KBB + cblk * 8192;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int t = 8 * rg + r;
+      const uint32_t koff = (uint32_t)t * 128 + (cpos ^ ((uint32_t)(t & 7) << 4));
+      const uint32_t kraw = *reinterpret_cast<const uint32_t *>(kr + koff);
+      const uint32_t qraw = *reinterpret_cast<const uint32_t *>(qr + koff);
+      const float k0 = bf16_lo(kraw), k1 = bf16_hi(kraw);
+      const float fk = tFK[t], fq = tFQ[t], fa = tFA[t], fb = tFB[t];
+      *reinterpret_cast<uint32_t *>(kd + koff) = pack_bf16x2(k0 * fk, k1 * fk);
+      *reinterpret_cast<uint32_t *>(qd + koff) = pack_bf16x2(bf16_lo(qraw) * fq, bf16_hi(qraw) * fq);
+      *reinterpret_cast<uint32_t *>(ab + koff) = pack_bf16x2(k0 * fa, k1 * fa);
+      *reinterpret_cast<uint32_t *>(bb + koff) = pack_bf16x2(k0 * fb, k1 * fb);
+    }
+  }
+  __syncwarp();
+  mbar_wait(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);
+  tc_fence_after();
+
+  // ---- 5'. Gram readback: TMEM lane r < 64 is key row i = r, lane 64 + t query
+  //          row t; column j is key j.  Warp (quad, qtr) takes 32 rows and key
+  //          columns 16 qtr .. +15 (block J = qtr).  With the row term Gp_i
+  //          (keys) or G_t (queries):
+  //            w = raw beta_j e^{row - G_j}   (A_w beta, B_w beta)
+  //            e = raw beta_j e^{row - Gp_j} = w a_j   (A_e beta, B_e beta)
+  //          keys j < i, queries j <= t, rows past the chunk's length zero.
+  //          Left of the diagonal block the factor splits at E_J into a row
+  //          and a column factor, both <= 1; inside it each factor is one exp.
+  //          The same images and N as the per-channel path ----
+  {
+    const bool isQ = quad >= 2;
+    const int r = 32 * (quad & 1) + lane, J = qtr, I = r >> 4;
+    float *nae = reinterpret_cast<float *>(sX + X_NAE);
+    float w[16], e[16];
+    if (J <= 2 * (quad & 1) + 1) {  // warp-uniform: some row of the warp reaches block J
+      float v[16], cf[16], aj[16];
+      tmem_ld16(taddr(tm, 32 * quad, TM_GRAM + 16 * J), v);
+      const bool diag = J == I;
+#pragma unroll
+      for (int u = 0; u < 16; u += 4) {
+        // diagonal block: beta_j and G_j; left of it: beta_j e^{E_J - G_j}
+        const float4 c4 = *reinterpret_cast<const float4 *>((diag ? sBeta : tCW) + 16 * J + u);
+        const float4 a4 = *reinterpret_cast<const float4 *>(tA + 16 * J + u);
+        cf[u] = c4.x; cf[u + 1] = c4.y; cf[u + 2] = c4.z; cf[u + 3] = c4.w;
+        aj[u] = a4.x; aj[u + 1] = a4.y; aj[u + 2] = a4.z; aj[u + 3] = a4.w;
+      }
+      const float rowg = isQ ? tG[r] : tGp[r];
+      const bool rowok = r < L && J <= I;
+      const float rowf = (rowok && !diag) ? expf(rowg - tE[J]) : 0.f;
+      tmem_ld_wait();
+      if (diag) {
+        // keys: beta_j D[a][u]; queries: beta_j D[a][u] a_t for u < a, beta_t at u = a
+        const int a = r & 15;
+        const float4 *drow = reinterpret_cast<const float4 *>(tD + r * kLdD);
+        const float rf = !rowok ? 0.f : isQ ? tA[r] : 1.f;
+#pragma unroll
+        for (int q4 = 0; q4 < 4; ++q4) {
+          const float4 d4 = drow[q4];
+          const float dd[4] = {d4.x, d4.y, d4.z, d4.w};
+#pragma unroll
+          for (int k4 = 0; k4 < 4; ++k4) {
+            const int u = 4 * q4 + k4;
+            const float f = (isQ && u == a) ? (rowok ? 1.f : 0.f) : dd[k4] * rf;
+            w[u] = v[u] * cf[u] * f;
+            e[u] = w[u] * aj[u];
+          }
+        }
+      } else {
+#pragma unroll
+        for (int u = 0; u < 16; ++u) {
+          w[u] = v[u] * rowf * cf[u];
+          e[u] = w[u] * aj[u];
+        }
+      }
+    } else {
+#pragma unroll
+      for (int u = 0; u < 16; ++u) w[u] = e[u] = 0.f;
+    }
+    const int row_w = isQ ? 64 + r : r;
+#pragma unroll
+    for (int hseg = 0; hseg < 2; ++hseg) {
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = w[8 * hseg + u];
+      st16(sX + X_AWBW + kmajor_off(row_w, 16 * J + 8 * hseg), pack8(x));
+    }
+    if (!isQ) {
+      if (J <= I) {  // T^{-1} reads N only on and below the diagonal blocks
+#pragma unroll
+        for (int u = 0; u < 16; u += 4)
+          *reinterpret_cast<float4 *>(nae + r * LDN + 16 * J + u) =
+              make_float4(e[u], e[u + 1], e[u + 2], e[u + 3]);
+      }
+    } else {
+#pragma unroll
+      for (int hseg = 0; hseg < 2; ++hseg) {
+        float x[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) x[u] = e[8 * hseg + u];
+        st16(sX + X_BE + kmajor_off(r, 16 * J + 8 * hseg), pack8(x));
+      }
+    }
+  }
+  fence_async_smem();  // the images are operands of the next products
+  __syncthreads();
+  }  // scalar gate
 
   // ---- 6. products that need no T^{-1}, issued before it is built:
   //         Y^T = V^T (A_w beta)^T;  O_intra = tril(B_w) beta V (rows t < 64 of an
@@ -826,7 +1042,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (tid == 0) {
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_W, desc_mnmajor(smem_u32(sK), 16 * kk, 8192),
+      mma_bf16(tm + TM_W, desc_mnmajor(smem_u32(sKd), 16 * kk, 8192),
                desc_kmajor(smem_u32(sX + X_TINVB), 16 * kk, 0), idesc_bf16(128, 64, true, false),
                kk > 0);
     mma_commit(bar_mma);
@@ -928,7 +1144,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const int t = 16 * qtr + 8 * seg + u;
-        const float qg = ld_bf16(sQ, (c >> 6) * 8192 + kmajor_off(t, c & 63));  // q e^{G}
+        const float qg = ld_bf16(sQd, (c >> 6) * 8192 + kmajor_off(t, c & 63));  // q e^{G}
         x[u] = (t < L) ? qg - x16[8 * seg + u] : 0.f;
       }
       st16(sX + X_QPI + sw128((uint32_t)(c * 128 + (16 * qtr + 8 * seg) * 2)), pack8(x));

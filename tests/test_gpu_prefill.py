@@ -73,6 +73,34 @@ def test_gdn_shared_heads(io):
     _check(W.make_prefill(w, seed=6))
 
 
+@pytest.mark.parametrize("gate,scale", [("channel", 1.0), ("scalar", 1.0), ("scalar", 4.0)])
+def test_strong_decay(gate, scale):
+    """Strong gates: a per-token log-decay of about -0.7 x scale (up to ~ -5 x
+    scale), so in-chunk cumulative decays reach e^{-40 scale} and the factors
+    taken at a token and at the token before it differ by e^{g}, far beyond the
+    tolerance.  The per-channel path's sub-chunk anchors and the scalar path's
+    elementwise factors both have to keep every product finite and right."""
+    base = "kda_prefill" if gate == "channel" else "gdn_long"
+    w = W.WORKLOADS[base].replace(T=200, H_qk=2, H_v=2 if gate == "channel" else 4,
+                                  gate_scale=scale, init_state=True)
+    _check(W.make_prefill(w, seed=13))
+
+
+def test_gdn_packed_sequences():
+    """Scalar gate, packed sequences (empty, one-token, chunk-aligned and
+    ragged): a chunk's rows past its length hold the next sequence's tokens."""
+    w = W.WORKLOADS["gdn_long"].replace(H_qk=2, H_v=4, init_state=True, gate_scale=0.5)
+    _check(W.make_prefill(w, seed=14, lengths=[70, 0, 1, 128, 0, 200, 63, 65]))
+
+
+def test_gdn_dense_batch_ragged_tail():
+    """Scalar gate, B = 3 dense sequences of 100 tokens: each sequence's last
+    chunk reads the next sequence's first 28 tokens as its rows 36..63."""
+    w = W.WORKLOADS["gdn_long"].replace(B=3, T=100, H_qk=2, H_v=4, init_state=True,
+                                        gate_scale=0.5)
+    _check(W.make_prefill(w, seed=15))
+
+
 def test_no_initial_state_no_final_state():
     import torch
     import gated_delta_rule_87_b200 as gdr
