@@ -261,11 +261,12 @@ constexpr uint32_t X_OII = 16384;     // after the last products: O_intra image 
 constexpr uint32_t X_QCI = 32768;     // after the last products: Qc image (32 KB)
 
 // TMEM columns (W, Y die at their readback, U at its readback)
-// Rounds of products: the Gram; Y and the first O_intra term (issued before
-// T^{-1} is built, which needs neither); W and U; then P and X (one thread)
-// beside the second O_intra term and Qc (another).
+// Rounds of products: the Gram; Y, the first O_intra term and the first Qc
+// term (issued before T^{-1} is built, which none of them needs; the last
+// products that read v); W and U; then P and X (one thread) beside the second
+// O_intra and Qc terms (another).
 constexpr uint32_t TM_GRAM = 0, TM_Y = 320, TM_OI = 128, TM_W = 256, TM_U = 0, TM_P = 0,
-                   TM_QC = 256, TM_X = 384;
+                   TM_QC = 384, TM_X = 256;
 
 __device__ __forceinline__ float ld_bf16(const unsigned char *base, uint32_t off) {
   return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(base + off));
@@ -402,9 +403,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // Items' chunk-table entries are read one item ahead of their use, so no
   // thread waits on a global load between phases.
   auto entry = [&](int w) { return w < total ? chunks.entry(w / H_v) : ChunkEntry{0, 0, 0, 0}; };
-  // g is loaded as soon as the previous item has taken its decays (its bytes
-  // join the phase without an arrival); q, k and v when the previous item is
-  // done with them (the arrival).  Thread 0.
+  // Each tile of the next item loads as soon as the current one is done with
+  // its buffer: g once the decays are taken, v once the products before T^{-1}
+  // have run, q and k once their last reader has run (the raw-tile Gram and
+  // the image pass with a scalar gate, before v; Q' with a per-channel gate,
+  // after v).  Every load but the last adds its bytes to the phase without an
+  // arrival; the last one arrives, so the phase completes only when every tile
+  // has landed.  All from thread kIoThread, in program order.
   auto load_g = [&](int w, const ChunkEntry &e) {
     if (CHANNEL) {
       fence_async_smem();
@@ -412,17 +417,27 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       tma_load_3d(sG, &tm_g, 0, w % H_v, e.start, bar_tma);
     }
   };
-  auto load_qkv = [&](int w, const ChunkEntry &e) {
-    const int hh = w % H_v, hkk = hh / (H_v / H_qk);
-    const int ts = e.start;
+  auto load_qk = [&](int w, const ChunkEntry &e, bool arrive) {
+    const int hkk = (w % H_v) / (H_v / H_qk);
     fence_async_smem();
-    mbar_arrive_expect_tx(bar_tma, 3 * 16384);
+    if (arrive)
+      mbar_arrive_expect_tx(bar_tma, 2 * 16384);
+    else
+      mbar_expect_tx(bar_tma, 2 * 16384);
 #pragma unroll
     for (int cb = 0; cb < 2; ++cb) {
-      tma_load_3d(sQ + cb * QK_CB, &tm_q, cb * 64, hkk, ts, bar_tma);
-      tma_load_3d(sK + cb * QK_CB, &tm_k, cb * 64, hkk, ts, bar_tma);
-      tma_load_3d(sV + cb * 8192, &tm_v, cb * 64, hh, ts, bar_tma);
+      tma_load_3d(sQ + cb * QK_CB, &tm_q, cb * 64, hkk, e.start, bar_tma);
+      tma_load_3d(sK + cb * QK_CB, &tm_k, cb * 64, hkk, e.start, bar_tma);
     }
+  };
+  auto load_v = [&](int w, const ChunkEntry &e, bool arrive) {
+    fence_async_smem();
+    if (arrive)
+      mbar_arrive_expect_tx(bar_tma, 16384);
+    else
+      mbar_expect_tx(bar_tma, 16384);
+#pragma unroll
+    for (int cb = 0; cb < 2; ++cb) tma_load_3d(sV + cb * 8192, &tm_v, cb * 64, w % H_v, e.start, bar_tma);
   };
   auto prefetch_l2 = [&](int w, const ChunkEntry &e) {  // thread 0: a later item's tiles into L2
     const int ck = w / H_v, hh = w - ck * H_v, hkk = hh / (H_v / H_qk);
@@ -446,7 +461,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   ChunkEntry ce = entry(work), ce_next = entry(work + gridDim.x);
   if (tid == kIoThread) {
     load_g(work, ce);
-    load_qkv(work, ce);
+    load_v(work, ce, false);
+    load_qk(work, ce, true);
     if (work + (int)gridDim.x < total) prefetch_l2(work + gridDim.x, ce_next);
   }
   if (tid < C) load_beta(work, ce, nbeta, ngsc);
@@ -461,6 +477,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   if (tid < C) {
     sBeta[tid] = nbeta;
     if (!CHANNEL) sGsc[tid] = ngsc;
+    // the next item's, a whole item ahead of their use
+    if (next < total) load_beta(next, ce_next, nbeta, ngsc);
   }
   mbar_wait(bar_tma, it & 1, hdr, KDA_DEVICE_TIMEOUT);
   __syncthreads();
@@ -916,12 +934,15 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   fence_async_smem();  // the images are operands of the next products
   __syncthreads();
+  // the raw q, k tiles are consumed (Gram and image pass): the next item's load now
+  if (tid == kIoThread && next < total) load_qk(next, ce_next, false);
   }  // scalar gate
 
   // ---- 6. products that need no T^{-1}, issued before it is built:
   //         Y^T = V^T (A_w beta)^T;  O_intra = tril(B_w) beta V (rows t < 64 of an
   //         M = 128 product whose upper 64 rows read the bytes after the operand
-  //         and are discarded) ----
+  //         and are discarded);  Qc = (beta K e^{G_L-G})^T V.  With these v is
+  //         read for the last time ----
   if (tid == 256) {
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
@@ -934,6 +955,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_OI, desc_kmajor(smem_u32(sX + X_AWBW + 64 * 128), 16 * kk, 0),
                desc_mnmajor(smem_u32(sV), 16 * kk, 8192), idesc_bf16(128, 128, false, true),
+               kk > 0);
+#pragma unroll
+    for (int kk = 0; kk < 4; ++kk)
+      mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sm + OFF_KAB), 16 * kk, 8192),
+               desc_mnmajor(smem_u32(sV), 16 * kk, 8192), idesc_bf16(128, 128, true, true),
                kk > 0);
     mma_commit(bar_yo);
   }
@@ -1020,6 +1046,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   } else {
     // warps 8-15, meanwhile: Y (lanes n, cols i) -> K-major [n][t]
     mbar_wait(bar_yo, it & 1, hdr, KDA_DEVICE_TIMEOUT);
+    // the step-6 products were the last to read v: the next item's v tile now
+    if (tid == kIoThread && next < total) load_v(next, ce_next, !CHANNEL);
     tc_fence_after();
     const int cg = (warp >> 2) - 2;  // column group: 32 cg .. +31
     float v[32];
@@ -1082,7 +1110,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   // ---- 9. thread 32: K_b^T beta W (for P), X = W^T (B_e beta)^T (for Q');
   //         thread 0: O_intra -= tril(B_e) beta U (M = 128 as in step 6),
-  //         Qc = (beta K e^{G_L-G})^T V - (beta K e^{G_L-Gp})^T U (lanes i, columns j) ----
+  //         Qc -= (beta K e^{G_L-Gp})^T U (lanes i, columns j) ----
   if (tid == 32) {
     const uint32_t wsm = smem_u32(sX + X_W);
 #pragma unroll
@@ -1096,17 +1124,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mma_commit(bar_px);
   } else if (tid == 0) {
     const uint32_t usm = smem_u32(sX + X_U);
-    // the first O_intra term (thread 288) has completed: warps 8-15 passed bar_yo's
-    // phase before the barrier ahead of the W/U round
+    // the first O_intra and Qc terms (thread 288) have completed: warps 8-15
+    // passed bar_yo's phase before the barrier ahead of the W/U round
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_OI, desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0), desc_kmajor(usm, 16 * kk, 0),
                idesc_bf16(128, 128, false, false, true), 1);
-#pragma unroll
-    for (int kk = 0; kk < 4; ++kk)
-      mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sm + OFF_KAB), 16 * kk, 8192),
-               desc_mnmajor(smem_u32(sV), 16 * kk, 8192), idesc_bf16(128, 128, true, true),
-               kk > 0);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_QC, desc_mnmajor(smem_u32(sm + OFF_KBB), 16 * kk, 8192),
@@ -1158,12 +1181,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     bulk_s2g(slot + SLOT_P, sX + X_PI, 32768);
     bulk_s2g(slot + SLOT_QP, sX + X_QPI, 16384);
     bulk_commit();
+    if (CHANNEL && next < total) load_qk(next, ce_next, true);  // Q' has read the q tile
   }
   mbar_wait(bar_oq, it & 1, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
-  // the input tiles are consumed: start the next item's loads now
-  if (tid == kIoThread && next < total) load_qkv(next, ce_next);
-  if (tid < C && next < total) load_beta(next, ce_next, nbeta, ngsc);
   {
     // warp (quad, qtr) holds rows 32 quad + lane, value columns 32 qtr .. +31,
     // i.e. one row of column slice qtr
