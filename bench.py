@@ -226,6 +226,8 @@ def run_ours(args, world, rank, local):
                                 device_id=device)
     peaks = _peaks()
     w = W.WORKLOADS[args.workload]
+    if args.tokens is not None:
+        w = w.replace(T=args.tokens)
     x = W.make_prefill(w, seed=0)
     N = x.num_seqs
     T_total = x.total_tokens
@@ -302,7 +304,8 @@ def run_ours(args, world, rank, local):
     algo_flops = prefill_flops(w, T_total)
     kb = kernel_algo_bytes(dominant, w, T_total, N)
     achieved = kb / (kern_ms[dominant] / 1e3) / 1e9
-    traffic = measured_traffic(dominant, w.name)
+    # counters are per launch of the named workload at its own size
+    traffic = measured_traffic(dominant, w.name) if args.tokens is None else None
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": traffic, "peak_source": peaks["source"], "kernel": dominant,
@@ -501,7 +504,12 @@ def main():
                     choices=[k for k, v in W.WORKLOADS.items() if v.kind == "prefill"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="sequence length of a dense workload in place of its own "
+                         "(a smaller case of the same kernels, e.g. for a profiler capture)")
     args = ap.parse_args()
+    if args.tokens is not None and (W.WORKLOADS[args.workload].varlen or args.tokens < 1):
+        ap.error("--tokens takes a positive length and a dense workload")
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup()
     if args.impl == "reference":
