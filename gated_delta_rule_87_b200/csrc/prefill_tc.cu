@@ -1363,34 +1363,45 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
     }
   } else if (warp == kScanMmaWarp) {
     // ---------------- tensor-core issue ----------------
-    if (lane == 0) {
-      constexpr uint32_t idS = idesc_bf16(128, NS, false, true);  // P K-major, S MN-major
-      constexpr uint32_t idO = idesc_bf16(128, NS, true, true);   // Q' MN-major, S MN-major
-      for (int u = 0; u < nch; ++u) {
-        const int st = u % S, b = u & 1;
-        if (!mbar_wait(&full[st], (u / S) & 1, err, KDA_DEVICE_TIMEOUT)) break;
-        if (!mbar_wait(&sb_ready[b], (u >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
-        tc_fence_after();
-        const uint32_t stage = smem_u32(sm + st * Cfg::ST_BYTES);
-        const uint32_t sb = smem_u32(sm + Cfg::OFF_SB + b * Cfg::SB_BYTES);
+    // The whole warp runs the loop and computes the operand descriptors
+    // (warp-uniform values); one elected lane issues the products.
+    constexpr uint32_t idS = idesc_bf16(128, NS, false, true);  // P K-major, S MN-major
+    constexpr uint32_t idO = idesc_bf16(128, NS, true, true);   // Q' MN-major, S MN-major
+    for (int u = 0; u < nch; ++u) {
+      const int st = u % S, b = u & 1;
+      if (!mbar_wait_warp(&full[st], (u / S) & 1, err, KDA_DEVICE_TIMEOUT)) break;
+      if (!mbar_wait_warp(&sb_ready[b], (u >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
+      tc_fence_after();
+      const uint32_t stage = smem_u32(sm + st * Cfg::ST_BYTES);
+      const uint32_t sb = smem_u32(sm + Cfg::OFF_SB + b * Cfg::SB_BYTES);
+      uint64_t da[8], dbs[8];
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tm + Cfg::TD_S, desc_kmajor(stage + Cfg::ST_P, 16 * kk, 16384),
-                   sop_desc<NS>(sb, kk), idS, kk > 0);
+      for (int kk = 0; kk < 8; ++kk) {
+        da[kk] = desc_kmajor(stage + Cfg::ST_P, 16 * kk, 16384);
+        dbs[kk] = sop_desc<NS>(sb, kk);
+      }
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mma_bf16(tm + Cfg::TD_S, da[kk], dbs[kk], idS, kk > 0);
         mma_commit(ds_full);
-        if (u >= 2 && !mbar_wait(&do_free[b], ((u - 2) >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
-        tc_fence_after();
+      }
+      __syncwarp();
+      if (u >= 2 && !mbar_wait_warp(&do_free[b], ((u - 2) >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
+      tc_fence_after();
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          mma_bf16(tm + Cfg::TD_O + NS * b, desc_mnmajor(stage + Cfg::ST_QP, 16 * kk, 16384),
-                   sop_desc<NS>(sb, kk), idO, kk > 0);
+      for (int kk = 0; kk < 8; ++kk) da[kk] = desc_mnmajor(stage + Cfg::ST_QP, 16 * kk, 16384);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mma_bf16(tm + Cfg::TD_O + NS * b, da[kk], dbs[kk], idO, kk > 0);
         mma_commit(&do_full[b]);
         mma_commit(&empty[st]);
       }
-      // every issued product has finished before TMEM is released
-      mma_commit(drain);
-      mbar_wait(drain, 0, err, KDA_DEVICE_TIMEOUT);
+      __syncwarp();
     }
+    // every issued product has finished before TMEM is released
+    if (elect_one()) mma_commit(drain);
+    __syncwarp();
+    mbar_wait_warp(drain, 0, err, KDA_DEVICE_TIMEOUT);
   } else if (warp < 4) {
     // ---------------- the state chain: row i, NS columns ----------------
     const int i = 32 * warp + lane;

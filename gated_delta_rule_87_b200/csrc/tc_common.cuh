@@ -50,6 +50,18 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
                : "memory");
 }
 
+// One lane of a converged warp (elect.sync): the issuing lane for tensor-core
+// work whose operands the whole warp computed (warp-uniform values).
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "elect.sync _|p, 0xffffffff;\n\t"
+      "selp.b32 %0, 1, 0, p;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
@@ -98,6 +110,13 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, int32_
     if (mbar_try_wait(bar, parity)) return true;
   if (err) atomicExch(err, code);
   return false;
+}
+
+// mbar_wait by all 32 lanes of a warp, with one verdict for the whole warp
+// (the warp stays converged for the .sync.aligned instructions that follow).
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t *bar, uint32_t parity, int32_t *err,
+                                               int32_t code) {
+  return __all_sync(0xffffffffu, mbar_wait(bar, parity, err, code));
 }
 
 // ---------------------------------------------------------------------------
