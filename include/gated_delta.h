@@ -294,7 +294,8 @@ KDA_API kda_status_t kda_check_device_status(const void *workspace, void *stream
 
 /* Diagnostic: runs one on-device wait that nothing ever completes, bounded like
  * every wait in the library's kernels (an mbarrier poll loop of at most
- * max_polls polls, each at most ~1 ms).  When the bound expires the kernel
+ * max_polls polls; a poll of a phase that never completes returns after a few
+ * microseconds on B200).  When the bound expires the kernel
  * writes KDA_DEVICE_TIMEOUT into the status word at the start of `workspace`
  * (any prefill workspace, or 4 bytes of device memory) and returns, exactly as
  * an expired wait inside a prefill does; kda_check_device_status() then
