@@ -300,24 +300,39 @@ __device__ __forceinline__ uint32_t to_tf32(float x) {
 }
 
 // d (16x8 fp32, per-lane fragment) += A[0..16)[k] * B[k][n0 .. n0+8) over k in [k_lo, k_hi)
-// (multiples of 8).  A and B are row-major fp32 in shared memory with row
-// strides lda, ldb; A points at row 0 / column 0 of the tile, B at row 0 and
-// column n0 is given separately.  Fragments follow the m16n8k8 layout: lane =
-// 4 g + t holds A (g, t), (g+8, t), (g, t+4), (g+8, t+4), B (t, g), (t+4, g) and
-// D (g, 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1).
+// (multiples of 8, at most 8 NSTEP).  A and B are row-major fp32 in shared
+// memory with row strides lda, ldb; A points at row 0 / column 0 of the tile,
+// B at row 0 and column n0 is given separately.  Fragments follow the
+// m16n8k8 layout: lane = 4 g + t holds A (g, t), (g+8, t), (g, t+4), (g+8, t+4),
+// B (t, g), (t+4, g) and D (g, 2t), (g, 2t+1), (g+8, 2t), (g+8, 2t+1).  The
+// k-steps are unrolled: every operand load of the first 8 NSTEP columns of A
+// and rows of B (all inside the tiles) is issued up front, and only the
+// products of steps in [k_lo, k_hi) run (a warp-uniform test), so no load
+// waits on the previous product.
+template <int NSTEP>
 __device__ __forceinline__ void warp_mma_tf32_range(float (&d)[4], const float *A, int lda,
                                                     const float *B, int ldb, int n0, int k_lo,
                                                     int k_hi, int lane) {
   const int g = lane >> 2, t = lane & 3;
-  for (int k0 = k_lo; k0 < k_hi; k0 += 8) {
-    const uint32_t a0 = to_tf32(A[g * lda + k0 + t]), a1 = to_tf32(A[(g + 8) * lda + k0 + t]);
-    const uint32_t a2 = to_tf32(A[g * lda + k0 + t + 4]), a3 = to_tf32(A[(g + 8) * lda + k0 + t + 4]);
-    const uint32_t b0 = to_tf32(B[(k0 + t) * ldb + n0 + g]), b1 = to_tf32(B[(k0 + t + 4) * ldb + n0 + g]);
+  uint32_t a[NSTEP][4], b[NSTEP][2];
+#pragma unroll
+  for (int s = 0; s < NSTEP; ++s) {
+    const int k0 = 8 * s;
+    a[s][0] = to_tf32(A[g * lda + k0 + t]);
+    a[s][1] = to_tf32(A[(g + 8) * lda + k0 + t]);
+    a[s][2] = to_tf32(A[g * lda + k0 + t + 4]);
+    a[s][3] = to_tf32(A[(g + 8) * lda + k0 + t + 4]);
+    b[s][0] = to_tf32(B[(k0 + t) * ldb + n0 + g]);
+    b[s][1] = to_tf32(B[(k0 + t + 4) * ldb + n0 + g]);
+  }
+#pragma unroll
+  for (int s = 0; s < NSTEP; ++s) {
+    if (8 * s < k_lo || 8 * s >= k_hi) continue;
     asm volatile(
         "mma.sync.aligned.m16n8k8.row.col.f32.tf32.tf32.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, "
         "{%8, %9}, {%0, %1, %2, %3};"
         : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+        : "r"(a[s][0]), "r"(a[s][1]), "r"(a[s][2]), "r"(a[s][3]), "r"(b[s][0]), "r"(b[s][1]));
   }
 }
 
@@ -325,7 +340,7 @@ __device__ __forceinline__ void warp_mma_tf32_range(float (&d)[4], const float *
 template <int K>
 __device__ __forceinline__ void warp_mma_tf32(float (&d)[4], const float *A, int lda, const float *B,
                                               int ldb, int lane) {
-  warp_mma_tf32_range(d, A, lda, B, ldb, 0, 0, K, lane);
+  warp_mma_tf32_range<K / 8>(d, A, lda, B, ldb, 0, 0, K, lane);
 }
 
 // Writes a 16x8 fp32 fragment to row-major shared memory at P (row stride ld).
@@ -1021,12 +1036,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const int m0 = 16 * (warp >> 2), n0 = 8 * (warp & 3);
       float d[4] = {0.f, 0.f, 0.f, 0.f};
       // tmp = N[32..63][0..31] T^{-1}[0..31][0..31]: rows k < n0 of the right factor are 0
-      warp_mma_tf32_range(d, nae + (32 + m0) * LDN, LDN, tinv, LDN, n0, n0 & ~7, 32, lane);
+      warp_mma_tf32_range<4>(d, nae + (32 + m0) * LDN, LDN, tinv, LDN, n0, n0 & ~7, 32, lane);
       store_frag(tmp + m0 * LDT + n0, LDT, d, lane);
       named_bar_sync(kTinvBar, kTinvThreads);
       float e[4] = {0.f, 0.f, 0.f, 0.f};
       // T^{-1}[32..63][32..63] tmp: columns k >= m0 + 16 of the left factor are 0
-      warp_mma_tf32_range(e, tinv + (32 + m0) * LDN + 32, LDN, tmp, LDT, n0, 0, m0 + 16, lane);
+      warp_mma_tf32_range<4>(e, tinv + (32 + m0) * LDN + 32, LDN, tmp, LDT, n0, 0, m0 + 16, lane);
       e[0] = -e[0]; e[1] = -e[1]; e[2] = -e[2]; e[3] = -e[3];
       store_frag(tinv + (32 + m0) * LDN + n0, LDN, e, lane);
     }
