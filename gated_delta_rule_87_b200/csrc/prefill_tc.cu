@@ -1351,7 +1351,9 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
   if (warp == kScanLoadWarp) {
     // ---------------- loads ----------------
     if (lane == 0) {
-      constexpr int kAhead = 4;  // chunks prefetched into L2 ahead of their stage load
+      // chunks prefetched into L2 ahead of their stage load: 2 measured best
+      // (further ahead, many chains' prefetches evict each other from L2)
+      constexpr int kAhead = 2;
       auto prefetch = [&](int u) {
         const unsigned char *src = slot_of(u);
         bulk_prefetch_l2(src + SLOT_P, 49152);  // P and Q'
