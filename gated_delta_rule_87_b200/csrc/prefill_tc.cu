@@ -837,26 +837,34 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // ---- 3'. while the Gram runs: the row-scaled tiles the later products read,
   //          in the per-channel path's layout: k e^{Gp} and q e^{G} (in the g
   //          buffer, which a scalar gate does not use), beta k e^{G_L - G} and
-  //          beta k e^{G_L - Gp}.  Thread: channel pair c2, rows 8 rg .. +7; a
-  //          warp covers one 128-byte row segment ----
+  //          beta k e^{G_L - Gp}.  Thread: channels c4 .. c4 + 3 (8 bytes,
+  //          inside one swizzled 16-byte chunk), rows 4 rg .. +3; a warp covers
+  //          one whole 256-byte row ----
   {
-    const int c2 = (tid & 63) * 2, rg = tid >> 6;
-    const uint32_t cblk = (uint32_t)(c2 >> 6), cpos = (uint32_t)(c2 & 63) * 2;
+    const int c4 = (tid & 31) * 4, rg = tid >> 5;
+    const uint32_t cblk = (uint32_t)(c4 >> 6), cpos = (uint32_t)(c4 & 63) * 2;
     const unsigned char *const kr = sK + cblk * QK_CB, *const qr = sQ + cblk * QK_CB;
     unsigned char *const kd = sm + OFF_G + cblk * 8192, *const qd = sm + OFF_G + 16384 + cblk * 8192;
     unsigned char *const ab = sm + OFF_KAB + cblk * 8192, *const bb = sm + OFF_KBB + cblk * 8192;
+    auto scaled = [](float2 x0, float2 x1, float f) {
+      const float2 ff = make_float2(f, f);
+      const float2 y0 = __fmul2_rn(x0, ff), y1 = __fmul2_rn(x1, ff);
+      return make_uint2(pack_bf16x2(y0.x, y0.y), pack_bf16x2(y1.x, y1.y));
+    };
 #pragma unroll
-    for (int r = 0; r < 8; ++r) {
-      const int t = 8 * rg + r;
+    for (int r = 0; r < 4; ++r) {
+      const int t = 4 * rg + r;
       const uint32_t koff = (uint32_t)t * 128 + (cpos ^ ((uint32_t)(t & 7) << 4));
-      const uint32_t kraw = *reinterpret_cast<const uint32_t *>(kr + koff);
-      const uint32_t qraw = *reinterpret_cast<const uint32_t *>(qr + koff);
-      const float k0 = bf16_lo(kraw), k1 = bf16_hi(kraw);
-      const float fk = tFK[t], fq = tFQ[t], fa = tFA[t], fb = tFB[t];
-      *reinterpret_cast<uint32_t *>(kd + koff) = pack_bf16x2(k0 * fk, k1 * fk);
-      *reinterpret_cast<uint32_t *>(qd + koff) = pack_bf16x2(bf16_lo(qraw) * fq, bf16_hi(qraw) * fq);
-      *reinterpret_cast<uint32_t *>(ab + koff) = pack_bf16x2(k0 * fa, k1 * fa);
-      *reinterpret_cast<uint32_t *>(bb + koff) = pack_bf16x2(k0 * fb, k1 * fb);
+      const uint2 kraw = *reinterpret_cast<const uint2 *>(kr + koff);
+      const uint2 qraw = *reinterpret_cast<const uint2 *>(qr + koff);
+      const float2 k0 = make_float2(bf16_lo(kraw.x), bf16_hi(kraw.x));
+      const float2 k1 = make_float2(bf16_lo(kraw.y), bf16_hi(kraw.y));
+      const float2 q0 = make_float2(bf16_lo(qraw.x), bf16_hi(qraw.x));
+      const float2 q1 = make_float2(bf16_lo(qraw.y), bf16_hi(qraw.y));
+      *reinterpret_cast<uint2 *>(kd + koff) = scaled(k0, k1, tFK[t]);
+      *reinterpret_cast<uint2 *>(qd + koff) = scaled(q0, q1, tFQ[t]);
+      *reinterpret_cast<uint2 *>(ab + koff) = scaled(k0, k1, tFA[t]);
+      *reinterpret_cast<uint2 *>(bb + koff) = scaled(k0, k1, tFB[t]);
     }
   }
   __syncwarp();
