@@ -531,8 +531,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
           g0 = g1 = sGsc[t];
         }
       }
-      a0[r] = expf(g0);
-      a1[r] = expf(g1);
+      a0[r] = __expf(g0);  // the intrinsic: its error is far below the bf16 rounding of every operand
+      a1[r] = __expf(g1);
       s0 += g0;
       s1 += g1;
       p0 *= a0[r];
@@ -583,7 +583,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         ge1 *= sPblk[J * DK + c2 + 1];
       }
     }
-    const float inv0 = expf(-sGsum[bI * DK + c2]), inv1 = expf(-sGsum[bI * DK + c2 + 1]);  // 1/PB_I
+    const float inv0 = __expf(-sGsum[bI * DK + c2]), inv1 = __expf(-sGsum[bI * DK + c2 + 1]);  // 1/PB_I
     float fa0 = 1.f, fa1 = 1.f;  // anchor E_0
     if (bI == 0) {
       fa0 = inv0;
