@@ -454,7 +454,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
     for (int cb = 0; cb < 2; ++cb) tma_load_3d(sV + cb * 8192, &tm_v, cb * 64, w % H_v, e.start, bar_tma);
   };
-  auto prefetch_l2 = [&](int w, const ChunkEntry &e) {  // thread 0: a later item's tiles into L2
+  auto prefetch_l2 = [&](int w, const ChunkEntry &e) {  // kIoThread: a later item's tiles into L2
     const int ck = w / H_v, hh = w - ck * H_v, hkk = hh / (H_v / H_qk);
     const int ts = e.start;
     (void)ck;
