@@ -114,3 +114,39 @@ def test_one_pass_decode_readout_equals_the_updated_state_read():
                                     threads=1)
         np.testing.assert_allclose(o, ro[0, 0], rtol=1e-12, atol=1e-12)
         np.testing.assert_allclose(S_new, rs[0, 0], rtol=1e-12, atol=1e-12)
+
+
+@pytest.mark.parametrize("scale", [0.05, 1.0, 4.0])
+def test_scalar_gate_gram_factorisation(scale):
+    """With one gate value per token the Grams are the raw dot products times
+    factors that are all <= 1: left of the diagonal 16-token block, a row factor
+    e^{row - E_J} times a column factor e^{E_J - G_j} (E_J: G at the end of key
+    block J); inside it, the product of the decays a_s of the tokens strictly
+    between the pair; the erase Grams are the write Grams times a_j."""
+    rng = np.random.default_rng(17)
+    C, d_k = 64, 8
+    q = rng.standard_normal((C, d_k))
+    k = rng.standard_normal((C, d_k))
+    g = -scale * np.log1p(np.exp(rng.standard_normal(C)))  # -scale * softplus(N)
+    G = np.cumsum(g)
+    Gp = G - g
+    a = np.exp(g)
+    E = G[15::16]
+    KK, QK = k @ k.T, q @ k.T
+    Aw = np.zeros((C, C)); Bw = np.zeros((C, C))
+    for r in range(C):
+        for j in range(C):
+            I, J = r // 16, j // 16
+            if J < I:
+                Aw[r, j] = KK[r, j] * np.exp(Gp[r] - E[J]) * np.exp(E[J] - G[j])
+                Bw[r, j] = QK[r, j] * np.exp(G[r] - E[J]) * np.exp(E[J] - G[j])
+            elif J == I:
+                d = np.prod(a[j + 1:r]) if j < r else 0.0  # e^{Gp_r - G_j}
+                Aw[r, j] = KK[r, j] * d
+                Bw[r, j] = QK[r, j] * (d * a[r] if j < r else (1.0 if j == r else 0.0))
+    Ae, Be = Aw * a[None, :], Bw * a[None, :]
+    lower, incl = np.tril(np.ones((C, C)), -1), np.tril(np.ones((C, C)))
+    np.testing.assert_allclose(Aw, KK * np.exp(Gp[:, None] - G[None, :]) * lower, rtol=1e-12, atol=1e-300)
+    np.testing.assert_allclose(Ae, KK * np.exp(Gp[:, None] - Gp[None, :]) * lower, rtol=1e-12, atol=1e-300)
+    np.testing.assert_allclose(Bw, QK * np.exp(G[:, None] - G[None, :]) * incl, rtol=1e-12, atol=1e-300)
+    np.testing.assert_allclose(Be, QK * np.exp(G[:, None] - Gp[None, :]) * incl, rtol=1e-12, atol=1e-300)
