@@ -125,7 +125,9 @@ KDA_API size_t kda_chunk_fwd_workspace_size(int32_t B, int32_t T, int32_t H, int
  * H_v % H_qk == 0 and v-head h reading q/k head h / (H_v / H_qk).
  *
  *   q, k [B, T, H_qk, d_k]; v, o [B, T, H_v, d_v]; g, beta [B, T, H_v];
- *   states [N, H_v, d_k, d_v].  Everything else as kda_chunk_fwd.
+ *   states [N, H_v, d_k, d_v].  Everything else as kda_chunk_fwd, except that
+ *   g has no lower bound here: with one gate value per token every scale
+ *   factor of the computation is at most 1.
  * ------------------------------------------------------------------------ */
 KDA_API kda_status_t gdn_chunk_fwd(const void *q, const void *k, const void *v, const float *g,
                            const float *beta, void *o, const float *initial_state,
