@@ -319,18 +319,6 @@ __device__ __forceinline__ void mma_bf16(uint32_t d_tmem, uint64_t a_desc, uint6
       : "memory");
 }
 
-// D[tmem] (+)= A[tmem] * B[smem]: A is M x 16 bf16 per instruction, row m in
-// TMEM lane m, element pairs (2c, 2c+1) packed in column c (low half first).
-__device__ __forceinline__ void mma_bf16_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
-                                            uint32_t idesc, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}"
-      ::"r"(d_tmem), "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
-      : "memory");
-}
-
 // Arrive on `bar` once every tcgen05 op issued so far by this thread is done.
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
   asm volatile(
@@ -357,12 +345,8 @@ __device__ __forceinline__ uint64_t desc_kmajor(uint32_t tile_saddr, int k0, uin
 }
 
 // MN-major SW128 tile: K rows of 64 MN-elements (128 bytes) each, per 64-wide
-// MN block; MN blocks `mn_block_bytes` apart.  Element (k, m) at:
-__device__ __forceinline__ uint32_t mnmajor_off(int k, int m, uint32_t mn_block_bytes) {
-  return (uint32_t)(m >> 6) * mn_block_bytes + sw128((uint32_t)(k * 128 + (m & 63) * 2));
-}
-
-// Descriptor for an MMA reading K rows [k0, k0 + 16) of an MN-major tile.
+// MN block; MN blocks `mn_block_bytes` apart.  Descriptor for K rows
+// [k0, k0 + 16):
 __device__ __forceinline__ uint64_t desc_mnmajor(uint32_t tile_saddr, int k0,
                                                  uint32_t mn_block_bytes) {
   return make_desc_sw128(tile_saddr + (uint32_t)k0 * 128, mn_block_bytes, 1024);
