@@ -86,6 +86,12 @@ def test_strong_decay(gate, scale):
     _check(W.make_prefill(w, seed=13))
 
 
+def test_gdn_unshared_heads():
+    """Scalar gate with as many q/k heads as v heads (no sharing), ragged length."""
+    w = W.WORKLOADS["gdn_long"].replace(T=150, H_qk=3, H_v=3, init_state=True, gate_scale=0.3)
+    _check(W.make_prefill(w, seed=16))
+
+
 def test_gdn_packed_sequences():
     """Scalar gate, packed sequences (empty, one-token, chunk-aligned and
     ragged): a chunk's rows past its length hold the next sequence's tokens."""
