@@ -2,13 +2,15 @@
 """Benchmark of the gated delta-rule hot path on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
-                    [--workload kda_prefill] [--no-decode] [--no-cpu-baseline]
+                    [--workload kda_prefill] [--no-decode] [--no-cpu-baseline] [--no-extra]
 
 One step = one KDA prefill call (``kda_chunk_fwd``) over the whole synthetic
 workload (B=1, H=32, T=4096, d_k=d_v=128, bf16 q/k/v, fp32 gate/beta/state),
 inputs resident in HBM.  The same JSON line also carries the decode-step
 measurement (256 sequences x 32 heads, state updated in place, 64 steps) as
-``decode``.  L2 (126 MB) is flushed by writing a 256 MB buffer before every
+``decode``, and the other timed prefill configurations (8 packed KDA sequences;
+Gated DeltaNet T=65536 with 16 q/k and 32 v heads) as ``prefill_configs``,
+each with its own rooflines.  L2 (126 MB) is flushed by writing a 256 MB buffer before every
 timed call.  Times are CUDA-event device times on the launching stream; with
 N > 1 ranks every rank runs its own copy of the workload (weak scaling, no
 data-path collective) and the slowest rank's time is reported.
@@ -215,7 +217,6 @@ def aggregate_throughput(units_per_rank: float, ms_max: float, world: int) -> fl
 # --------------------------------------------------------------------------- #
 def run_ours(args, world, rank, local):
     import torch
-    import gated_delta_rule_87_b200 as gdr
 
     device = torch.device("cuda", local)
     torch.cuda.set_device(device)
@@ -225,9 +226,71 @@ def run_ours(args, world, rank, local):
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=device)
     peaks = _peaks()
+    stream = torch.cuda.current_stream(device)
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     w = W.WORKLOADS[args.workload]
     if args.tokens is not None:
         w = w.replace(T=args.tokens)
+    main = bench_prefill(w, args, device, world, peaks, stream, flush, with_e2e=True,
+                         tokens_override=args.tokens is not None)
+
+    line = {
+        "metric": "KDA prefill tokens/s (decode-step state GB/s in 'decode'), % of roofline, 1xB200",
+        "value": main["value"], "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": main["ms_per_step"], "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": main["dtype"],
+        "data": "synthetic (seeded normals shaped like the workload)",
+        "config": main["config"],
+        "roofline": main["roofline"],
+        "call_roofline": main["call_roofline"],
+        "kernels": main["kernels"],
+        "e2e": main["e2e"],
+        "gpu_launches": main["launches"],
+        "clocks": main["clocks"],
+        "step_ms_min_max": main["step_ms_min_max"],
+    }
+    x_main = main.pop("_inputs")
+
+    if not args.no_decode:
+        line["decode"] = bench_decode(args, device, world, peaks, stream, flush)
+        line["gpu_launches"] += line["decode"]["launches"]
+
+    # the other timed prefill configurations, each with its own rooflines
+    if not args.no_extra and args.tokens is None:
+        extra = {}
+        for name in EXTRA_PREFILL:
+            if name == w.name:
+                continue
+            r = bench_prefill(W.WORKLOADS[name], args, device, world, peaks, stream, flush,
+                              with_e2e=False)
+            r.pop("_inputs")
+            line["gpu_launches"] += r.pop("launches")
+            extra[name] = r
+        line["prefill_configs"] = extra
+
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(x_main, w)
+
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier(device_ids=[device.index])
+        dist.destroy_process_group()
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+# prefill configurations timed besides the main one (their own sub-objects)
+EXTRA_PREFILL = ("kda_prefill", "kda_varlen", "gdn_long")
+
+
+def bench_prefill(w, args, device, world, peaks, stream, flush, with_e2e=False,
+                  tokens_override=False):
+    """Device-timed prefill calls on one workload (inputs resident in HBM, L2
+    flushed before every call), per-kernel times from the library's trace
+    events, rooflines, and optionally the end-to-end time through the public
+    API with host buffers."""
+    import torch
+    import gated_delta_rule_87_b200 as gdr
     x = W.make_prefill(w, seed=0)
     N = x.num_seqs
     T_total = x.total_tokens
@@ -244,7 +307,8 @@ def run_ours(args, world, rank, local):
     }
     if x.initial_state is not None:
         host["s0"] = f32(x.initial_state, x.initial_state.shape)
-    host = {k: v.pin_memory() for k, v in host.items()}
+    if with_e2e:
+        host = {k: v.pin_memory() for k, v in host.items()}
     dev = {k: v.to(device) for k, v in host.items()}
     cu = torch.from_numpy(x.cu_seqlens).to(device) if varlen else None
     s0 = dev.get("s0")
@@ -252,27 +316,25 @@ def run_ours(args, world, rank, local):
     sT = torch.empty((N, w.H_v, w.d_k, w.d_v), dtype=torch.float32, device=device)
     fn = gdr.kda_chunk_fwd if w.gate == "channel" else gdr.gdn_chunk_fwd
     ws = None
-    stream = torch.cuda.current_stream(device)
 
     def step(q, k, v, g, beta, s0_):
         nonlocal ws
         _, _, ws = fn(q, k, v, g, beta, s0_, cu, o=o, final_state=sT, workspace=ws)
 
-    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     for _ in range(args.warmup):
         flush.zero_()
         step(dev["q"], dev["k"], dev["v"], dev["g"], dev["beta"], s0)
     torch.cuda.synchronize()
     st, code = gdr.check_device_status(ws)
     if st != gdr.KDA_OK:
-        raise RuntimeError(f"device status {code}")
+        raise RuntimeError(f"{w.name}: device status {code}")
 
     # ---- device-timed steps (inputs resident) ----
     evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
            for _ in range(args.steps)]
     barrier(world, device)
     torch.cuda.synchronize()
-    with ClockSampler(local) as clocks:
+    with ClockSampler(device.index) as clocks:
         for i in range(args.steps):
             flush.zero_()
             evs[i][0].record(stream)
@@ -305,7 +367,7 @@ def run_ours(args, world, rank, local):
     kb = kernel_algo_bytes(dominant, w, T_total, N)
     achieved = kb / (kern_ms[dominant] / 1e3) / 1e9
     # counters are per launch of the named workload at its own size
-    traffic = measured_traffic(dominant, w.name) if args.tokens is None else None
+    traffic = measured_traffic(dominant, w.name) if not tokens_override else None
     roofline = {"bound": "hbm", "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
                 "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4),
                 "traffic": traffic, "peak_source": peaks["source"], "kernel": dominant,
@@ -318,70 +380,57 @@ def run_ours(args, world, rank, local):
                      "achieved_tflops": round(algo_flops / (ms_local / 1e3) / 1e12, 2),
                      "roofline_us": round(t_roof * 1e6, 2),
                      "frac": round(t_roof / (ms_local / 1e3), 4),
-                     "roofline_tokens_per_s": round(tokens / t_roof, 1)}
+                     "roofline_tokens_per_s": round(tokens / t_roof, 1),
+                     "traffic": {k: measured_traffic(k, w.name) if not tokens_override else None
+                                 for k in kern_ms}}
     kernels = {k: {"us": round(v * 1e3, 2), "launches_per_step": len(per_kernel[k]) // args.steps}
                for k, v in kern_ms.items()}
+    launches = gdr_launches_per_call(w, varlen) * args.steps
 
-    # ---- end to end through the public API: pinned host -> device, call, back ----
-    o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
-    sT_host = torch.empty(sT.shape, dtype=sT.dtype).pin_memory()
-    d_in = {k: torch.empty_like(v) for k, v in dev.items()}
-    h2d = sum(v.numel() * v.element_size() for v in host.values())
-    d2h = o.numel() * o.element_size() + sT.numel() * sT.element_size()
-    e2e_ev = []
-    for i in range(max(2, min(args.steps, 10)) + 1):
-        flush.zero_()
-        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        for k_, v_ in host.items():
-            d_in[k_].copy_(v_, non_blocking=True)
-        step(d_in["q"], d_in["k"], d_in["v"], d_in["g"], d_in["beta"], d_in.get("s0"))
-        o_host.copy_(o, non_blocking=True)
-        sT_host.copy_(sT, non_blocking=True)
-        b.record(stream)
-        if i > 0:  # first iteration is a warm-up
-            e2e_ev.append((a, b))
-    torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / len(e2e_ev)
-    e2e_ms = max_over_ranks(e2e_ms, world, device)
-
-    launches_per_step = gdr_launches_per_call(w, varlen)
-
-    line = {
-        "metric": "KDA prefill tokens/s (decode-step state GB/s in 'decode'), % of roofline, 1xB200",
-        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": args.steps,
-        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True,
-        "scaling": "weak", "vs_baseline": None, "dtype": "bf16" if w.io_dtype == "bf16" else "f32",
-        "data": "synthetic (seeded normals shaped like the workload)",
+    out = {
+        "workload": w.name, "description": w.description,
+        "value": round(value, 1), "unit": "tokens/s", "ms_per_step": round(ms, 4),
+        "dtype": "bf16" if w.io_dtype == "bf16" else "f32",
         "config": {"workload": w.name, "description": w.description, "B": B, "T": T,
                    "H_qk": w.H_qk, "H_v": w.H_v, "d_k": w.d_k, "d_v": w.d_v,
                    "num_seqs": N, "tokens": T_total, "chunk": 64,
                    "l2": "flushed (256 MB write) before every timed call",
                    "parallelism": f"replicas x{world}, no collective"},
-        "roofline": roofline,
-        "call_roofline": call_roofline,
-        "kernels": kernels,
-        "e2e": {"value": round(tokens * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
-                "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
-                "d2h_bytes_per_step": d2h},
-        "gpu_launches": launches_per_step * args.steps,
+        "roofline": roofline, "call_roofline": call_roofline, "kernels": kernels,
         "clocks": clocks.summary(),
         "step_ms_min_max": [round(min(per), 4), round(max(per), 4)],
+        "launches": launches, "_inputs": x,
     }
 
-    if not args.no_decode:
-        line["decode"] = bench_decode(args, device, world, peaks, stream, flush)
-        line["gpu_launches"] += line["decode"]["launches"]
-
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        line["cpu_baseline"] = cpu_baseline(x, w)
-
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier(device_ids=[device.index])
-        dist.destroy_process_group()
-    if rank == 0:
-        print(json.dumps(line), flush=True)
+    # ---- end to end through the public API: pinned host -> device, call, back ----
+    if with_e2e:
+        o_host = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+        sT_host = torch.empty(sT.shape, dtype=sT.dtype).pin_memory()
+        d_in = {k: torch.empty_like(v) for k, v in dev.items()}
+        h2d = sum(v.numel() * v.element_size() for v in host.values())
+        d2h = o.numel() * o.element_size() + sT.numel() * sT.element_size()
+        e2e_ev = []
+        for i in range(max(2, min(args.steps, 10)) + 1):
+            flush.zero_()
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            for k_, v_ in host.items():
+                d_in[k_].copy_(v_, non_blocking=True)
+            step(d_in["q"], d_in["k"], d_in["v"], d_in["g"], d_in["beta"], d_in.get("s0"))
+            o_host.copy_(o, non_blocking=True)
+            sT_host.copy_(sT, non_blocking=True)
+            b.record(stream)
+            if i > 0:  # first iteration is a warm-up
+                e2e_ev.append((a, b))
+        torch.cuda.synchronize()
+        e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev) / len(e2e_ev)
+        e2e_ms = max_over_ranks(e2e_ms, world, device)
+        out["e2e"] = {"value": round(tokens * world / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+                      "ms_per_step": round(e2e_ms, 4), "h2d_bytes_per_step": h2d,
+                      "d2h_bytes_per_step": d2h}
+    del dev, o, sT, ws
+    torch.cuda.empty_cache()
+    return out
 
 
 def gdr_launches_per_call(w: W.Workload, varlen: bool) -> int:
@@ -504,6 +553,8 @@ def main():
                     choices=[k for k, v in W.WORKLOADS.items() if v.kind == "prefill"])
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="time only the main workload (not the other prefill configurations)")
     ap.add_argument("--tokens", type=int, default=None,
                     help="sequence length of a dense workload in place of its own "
                          "(a smaller case of the same kernels, e.g. for a profiler capture)")
@@ -512,6 +563,9 @@ def main():
         ap.error("--tokens takes a positive length and a dense workload")
     args.warmup = max(args.warmup, 3)
     world, rank, local = dist_setup()
+    if args.gpus != world:
+        ap.error(f"--gpus {args.gpus} but WORLD_SIZE is {world}: launch N ranks with "
+                 "torch.distributed.run (one process per GPU)")
     if args.impl == "reference":
         run_reference(args, world, rank)
         return

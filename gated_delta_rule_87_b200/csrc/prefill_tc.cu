@@ -42,12 +42,13 @@
 //            triangular inverse, and writes P, Q', Qc, O_intra (bf16) into a
 //            workspace slot laid out as the scan's shared-memory operand
 //            images.
-//   scan  -- one CTA per (sequence, v-head), walking the chunks in order
-//            with the fp32 state in registers of 8 chain warps and its bf16
-//            transpose in TMEM as the A operand: per chunk one MMA
-//            (P S)^T = S^T P^T (128x128x128) and one o^T = S^T Q'^T
-//            (128x64x128), then S <- P S + Qc and o = Q' S + O_intra, with a
-//            load warp double-buffering the slots and 4 output warps.
+//   scan  -- one CTA per (sequence, v-head, 32- or 64-column slice of the
+//            state), walking the chunks in order: the fp32 state rows in
+//            registers of 4 chain warps, its bf16 copy in shared memory as
+//            the MN-major B operand; per chunk one MMA P S (M = 128, N = the
+//            slice width, K = 128) and one Q' S (M padded to 128), then
+//            S <- P S + Qc and o = Q' S + O_intra, with a load warp
+//            streaming the slots through 2-3 stages and 2 output warps.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -231,7 +232,7 @@ constexpr uint32_t MISC_GSC = 256;     // f32[64] scalar gate
 constexpr uint32_t MISC_PBLK = 512;    // f32[4][128] product of a over each sub-chunk
 constexpr uint32_t MISC_GSUM = 2560;   // f32[4][128] sum of g over each sub-chunk
 constexpr uint32_t MISC_GLE = 4608;    // f32[128] e^{G_L}
-constexpr uint32_t MISC_BAR = 5120;    // 5 x u64
+constexpr uint32_t MISC_BAR = 5120;    // 5 x u64; the drain barrier at +48
 constexpr uint32_t MISC_TSLOT = 5160;  // u32
 constexpr uint32_t MISC_XP = 6144;     // f32[4][2][128] product of a over each half sub-chunk
 constexpr uint32_t MISC_XS = 10240;    // f32[4][2][128] sum of g over each half sub-chunk
@@ -386,6 +387,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   uint64_t *bar_yo = bar_tma + 2;    // Y and the first O_intra term (two commits)
   uint64_t *bar_px = bar_tma + 3;    // P and X (one commit)
   uint64_t *bar_oq = bar_tma + 4;    // the second O_intra term and Qc (one commit)
+  uint64_t *bar_drain = bar_tma + 6;  // after an expired wait: every issuing thread's last MMAs
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + MISC_TSLOT);
 
   if (hdr[0] != KDA_DEVICE_OK) return;
@@ -407,6 +409,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mbar_init(bar_yo, 2);
     mbar_init(bar_px, 1);
     mbar_init(bar_oq, 1);
+    mbar_init(bar_drain, 4);
     mbar_fence_init();
   }
   tc_fence_before();
@@ -425,8 +428,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // after v).  Every load but the last adds its bytes to the phase without an
   // arrival; the last one arrives, so the phase completes only when every tile
   // has landed.  All from thread kIoThread, in program order.
+  // TMA phases armed by kIoThread (loads whose last one carried the arrival)
+  // and whether loads of a phase not yet armed are in flight: an aborted CTA
+  // completes and waits out every such phase before it exits.
+  int tma_armed = 0, tma_done = 0;
+  bool tma_partial = false;
   auto load_g = [&](int w, const ChunkEntry &e) {
     if (CHANNEL) {
+      tma_partial = true;
       fence_async_smem();
       mbar_expect_tx(bar_tma, 32768);
       tma_load_3d(sG, &tm_g, 0, w % H_v, e.start, bar_tma);
@@ -434,6 +443,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   };
   auto load_qk = [&](int w, const ChunkEntry &e, bool arrive) {
     const int hkk = (w % H_v) / (H_v / H_qk);
+    tma_armed += arrive ? 1 : 0;
+    tma_partial = !arrive;
     fence_async_smem();
     if (arrive)
       mbar_arrive_expect_tx(bar_tma, 2 * 16384);
@@ -446,6 +457,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   };
   auto load_v = [&](int w, const ChunkEntry &e, bool arrive) {
+    tma_armed += arrive ? 1 : 0;
+    tma_partial = !arrive;
     fence_async_smem();
     if (arrive)
       mbar_arrive_expect_tx(bar_tma, 16384);
@@ -482,7 +495,13 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   if (tid < C) load_beta(work, ce, nbeta, ngsc);
 
-  for (int it = 0; work < total; ++it, work += gridDim.x) {
+  // Every bounded wait below ANDs its verdict into `ok`; the block barriers
+  // after the waits take one CTA-wide verdict, and on a failure every thread
+  // leaves the work loop together (the status word already holds
+  // KDA_DEVICE_TIMEOUT), so an expired wait costs one bound, not one per item.
+  bool ok = true, aborted = false;
+  int it = 0;
+  for (; work < total; ++it, work += gridDim.x) {
   const int chunk = work / H_v, h = work - chunk * H_v;
   const int L = ce.len;
   unsigned char *slot = slots + ((size_t)chunk * H_v + h) * SLOT_BYTES;
@@ -495,8 +514,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // the next item's, a whole item ahead of their use
     if (next < total) load_beta(next, ce_next, nbeta, ngsc);
   }
-  mbar_wait(bar_tma, it & 1, hdr, KDA_DEVICE_TIMEOUT);
-  __syncthreads();
+  {
+    const bool landed = mbar_wait(bar_tma, it & 1, hdr, KDA_DEVICE_TIMEOUT);
+    ok &= landed;
+    if (landed) tma_done = it + 1;
+  }
+  if (__syncthreads_or(!ok)) { aborted = true; break; }
   // readbacks: warp (quad, qtr) reads TMEM lanes 32*quad .. +31, column quarter qtr
   const int quad = warp & 3, qtr = warp >> 2;
   const int lane_row = 32 * quad + lane;
@@ -682,7 +705,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mma_commit(bar_mma);
   }
   __syncwarp();
-  mbar_wait(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);
+  ok &= mbar_wait(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
 
   // ---- 5. Gram readback: masked, beta-scaled, into the next operands ----
@@ -742,7 +765,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   }
   fence_async_smem();  // the images are operands of the next products
-  __syncthreads();
+  if (__syncthreads_or(!ok)) { aborted = true; break; }
   } else {
   // ---- 2'. scalar gate: every decay factor is a per-token scalar, so the Gram
   //          products take the raw tiles and the factors are applied to the
@@ -868,7 +891,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   }
   __syncwarp();
-  mbar_wait(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);
+  ok &= mbar_wait(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
 
   // ---- 5'. Gram readback: TMEM lane r < 64 is key row i = r, lane 64 + t query
@@ -956,7 +979,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   }
   fence_async_smem();  // the images are operands of the next products
-  __syncthreads();
+  if (__syncthreads_or(!ok)) { aborted = true; break; }
   // the raw q, k tiles are consumed (Gram and image pass): the next item's load now
   if (tid == kIoThread && next < total) load_qk(next, ce_next, false);
   }  // scalar gate
@@ -1068,7 +1091,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   } else {
     // warps 8-15, meanwhile: Y (lanes n, cols i) -> K-major [n][t]
-    mbar_wait(bar_yo, it & 1, hdr, KDA_DEVICE_TIMEOUT);
+    ok &= mbar_wait(bar_yo, it & 1, hdr, KDA_DEVICE_TIMEOUT);
     // the step-6 products were the last to read v: the next item's v tile now
     if (tid == kIoThread && next < total) load_v(next, ce_next, !CHANNEL);
     tc_fence_after();
@@ -1086,7 +1109,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   fence_async_smem();
   tc_fence_before();
-  __syncthreads();
+  if (__syncthreads_or(!ok)) { aborted = true; break; }
   tc_fence_after();
 
   // ---- 8. W^T = (K e^{Gp})^T T^{-T};  U^T = Y^T T^{-T} ----
@@ -1106,7 +1129,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mma_commit(bar_mma);
   }
   __syncwarp();
-  mbar_wait(bar_mma, 1, hdr, KDA_DEVICE_TIMEOUT);
+  ok &= mbar_wait(bar_mma, 1, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
   {
     // W (lanes c, cols t) -> K-major [c][t]; U (lanes n, cols t) -> K-major [n][t]
@@ -1128,7 +1151,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   fence_async_smem();
   tc_fence_before();
-  __syncthreads();
+  if (__syncthreads_or(!ok)) { aborted = true; break; }
   tc_fence_after();
 
   // ---- 9. thread 32: K_b^T beta W (for P), X = W^T (B_e beta)^T (for Q');
@@ -1160,7 +1183,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mma_commit(bar_oq);
   }
   __syncwarp();
-  mbar_wait(bar_px, it & 1, hdr, KDA_DEVICE_TIMEOUT);
+  ok &= mbar_wait(bar_px, it & 1, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
   // P and Q' leave TMEM for the slot while the last products run (disjoint columns)
   {
@@ -1198,7 +1221,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   fence_async_smem();
   tc_fence_before();
-  __syncthreads();  // the P / Q' images are written
+  if (__syncthreads_or(!ok)) { aborted = true; break; }  // the P / Q' images are written
   tc_fence_after();
   if (tid == kIoThread) {  // P and Q' images -> workspace slot
     bulk_s2g(slot + SLOT_P, sX + X_PI, 32768);
@@ -1206,7 +1229,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     bulk_commit();
     if (CHANNEL && next < total) load_qk(next, ce_next, true);  // Q' has read the q tile
   }
-  mbar_wait(bar_oq, it & 1, hdr, KDA_DEVICE_TIMEOUT);
+  ok &= mbar_wait(bar_oq, it & 1, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
   {
     // warp (quad, qtr) holds rows 32 quad + lane, value columns 32 qtr .. +31,
@@ -1235,7 +1258,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   fence_async_smem();
   tc_fence_before();
-  __syncthreads();
+  if (__syncthreads_or(!ok)) { aborted = true; break; }
   tc_fence_after();
   if (tid == kIoThread) {  // Qc and O_intra images -> workspace slot
     bulk_s2g(slot + SLOT_QC, sX + X_QCI, 32768);
@@ -1246,6 +1269,23 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   ce_next = ce_next2;
   }  // work items
 
+  if (aborted) {
+    // Nothing may still write this CTA's shared memory or TMEM when it exits:
+    // the issuing threads' last products finish (a commit arrives once every
+    // earlier tcgen05 op of its thread is done), and every TMA phase kIoThread
+    // armed (or began to fill without arming) lands.  All waits stay bounded.
+    if (tid == 0 || tid == 32 || tid == 256 || tid == 288) mma_commit(bar_drain);
+    if (tid == kIoThread) {
+      if (tma_partial) {
+        mbar_arrive(bar_tma);
+        ++tma_armed;
+      }
+      // phases before tma_done were waited for at the top of their items
+      for (int ph = tma_done; ph < tma_armed; ++ph)
+        mbar_wait(bar_tma, ph & 1, hdr, KDA_DEVICE_TIMEOUT);
+    }
+    mbar_wait(bar_drain, 0, hdr, KDA_DEVICE_TIMEOUT);
+  }
   if (tid == kIoThread) bulk_wait0();
   tc_fence_before();
   __syncthreads();

@@ -271,10 +271,19 @@ KDA_API kda_status_t kda_state_scatter(const float *src, float *pool,
  *  - Problems whose kda_chunk_fwd_workspace_size() exceeds 64 MiB are
  *    rejected with KDA_ERR_WORKSPACE (kda_last_error() gives the sizes);
  *    use kda_chunk_fwd with a workspace for them.
- *  - Every device that loads the library keeps the 64 MiB until exit.
- *  - The first call on each device looks up the array's device address
- *    (cudaGetSymbolAddress) with that device current; make that first call
- *    before capturing the stream into a CUDA graph.
+ *  - The 64 MiB are reserved on a device when the library's module holding
+ *    the array is loaded there.  Under CUDA's default lazy module loading
+ *    that is the first call of this function on that device (with
+ *    CUDA_MODULE_LOADING=EAGER, when the library is loaded); the memory then
+ *    stays reserved until the process exits or the context is destroyed.  A
+ *    host whose pool claims the device's memory should make one call first:
+ *    a call with T = 0 computes nothing and only reserves the array.  If it
+ *    cannot be reserved the call returns KDA_ERR_CUDA (kda_last_error() says
+ *    why).
+ *  - The first call on each device (and the first after a device reset)
+ *    looks up the array's device address (cudaGetSymbolAddress) with that
+ *    device current; make that first call before capturing the stream into
+ *    a CUDA graph.
  *  - All calls on a device share the array and it keeps the last call's
  *    contents (each call resets its own status word).  Calls whose kernels
  *    overlap on the GPU (different streams or threads) race on it: order

@@ -24,3 +24,21 @@ def load_golden(name):
             key, val = line.split("=", 1)
             out[key.strip()] = [float(x) for x in val.split()]
     return out
+
+
+def pytest_terminal_summary(terminalreporter):
+    """Print the errors the parity tests measured (whole tensor, worst 64-token
+    block of a head, worst sequence, final state, worst single state)."""
+    try:
+        import parity
+    except ImportError:
+        return
+    if not parity.RECORDS:
+        return
+    tr = terminalreporter
+    tr.section("parity errors (relative L2 against the fp64 oracle)")
+    tr.write_line(f"{'case':64s} {'o':>9s} {'o block':>9s} {'o seq':>9s} {'state':>9s} "
+                  f"{'st worst':>9s} {'bound':>7s}")
+    for label, eo, eb, esq, es, esx, tol in parity.RECORDS:
+        tr.write_line(f"{label[:64]:64s} {eo:9.2e} {eb:9.2e} {esq:9.2e} {es:9.2e} {esx:9.2e} "
+                      f"{tol:7.0e}")

@@ -35,3 +35,13 @@ def test_stored_traffic_is_used_only_for_the_source_it_was_taken_from(tmp_path, 
     assert bench.measured_traffic("other", "w") is None
     src.write_text("// kernel source, changed\n")
     assert bench.measured_traffic("k", "w") is None
+
+
+def test_gpu_count_must_match_the_ranks():
+    """--gpus N without N ranks is refused before any device work (the bench
+    never reports a one-GPU number under an N-GPU label)."""
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--gpus", "8"],
+                       capture_output=True, text=True, timeout=300, env=env)
+    assert r.returncode == 2
+    assert "WORLD_SIZE" in r.stderr

@@ -3,7 +3,7 @@ import numpy as np
 import pytest
 
 from gated_delta_rule_87_b200 import workloads as W
-from parity import rel_l2, to_device, to_host, tol_for
+from parity import RECORDS, rel_l2, to_device, to_host, tol_for
 
 pytestmark = pytest.mark.gpu
 
@@ -79,9 +79,17 @@ def test_kda_decode_full_size_sampled():
     ro, rs = _oracle(x, chains)
     n_idx = [c[0] for c in chains]
     h_idx = [c[1] for c in chains]
-    assert rel_l2(o[:, n_idx, h_idx], ro) <= 2e-2
-    assert rel_l2(s[n_idx, h_idx], rs) <= 1e-4
     assert np.isfinite(o).all() and np.isfinite(s).all()
+    os_, ss = o[:, n_idx, h_idx], s[n_idx, h_idx]
+    eo, es = rel_l2(os_, ro), rel_l2(ss, rs)
+    # per chain: each sampled (sequence, head) over its 64 steps, and its state
+    ec = (np.linalg.norm(os_ - ro, axis=(0, 2)) / np.linalg.norm(ro, axis=(0, 2))).max()
+    esc = (np.linalg.norm((ss - rs).reshape(64, -1), axis=1)
+           / np.linalg.norm(rs.reshape(64, -1), axis=1)).max()
+    RECORDS.append(("test_kda_decode_full_size_sampled", eo, ec, ec, es, esc, 2e-2))
+    assert eo <= 2e-2 and ec <= 2e-2, (eo, ec)
+    assert es <= 1e-4 and esc <= 1e-4, (es, esc)
+    assert eo <= 1e-2  # regression bound near the measured error
 
 
 def test_decode_zero_batch_is_noop():
