@@ -232,8 +232,8 @@ constexpr uint32_t MISC_GSC = 256;     // f32[64] scalar gate
 constexpr uint32_t MISC_PBLK = 512;    // f32[4][128] product of a over each sub-chunk
 constexpr uint32_t MISC_GSUM = 2560;   // f32[4][128] sum of g over each sub-chunk
 constexpr uint32_t MISC_GLE = 4608;    // f32[128] e^{G_L}
-constexpr uint32_t MISC_BAR = 5120;    // 5 x u64; the drain barrier at +48
-constexpr uint32_t MISC_TSLOT = 5160;  // u32
+constexpr uint32_t MISC_BAR = 5120;    // 5 x u64; the drain barrier at +48, two failure flags at +56
+constexpr uint32_t MISC_TSLOT = 5160;  // u32; the exact-Gram flag at +4
 constexpr uint32_t MISC_XP = 6144;     // f32[4][2][128] product of a over each half sub-chunk
 constexpr uint32_t MISC_XS = 10240;    // f32[4][2][128] sum of g over each half sub-chunk
 constexpr uint32_t PREP_SMEM = OFF_MISC + 14336 + 1024;
@@ -248,6 +248,11 @@ constexpr uint32_t X_AWBW = 0;        // 16 KB K-major B [128 i'][64 j]
 constexpr uint32_t X_BE = 16384;      // 8 KB  K-major B [64 i][64 j]
 constexpr uint32_t X_TINVB = 24576;   // 8 KB  K-major B [64 i][64 j]; scratch before
 constexpr int LDN = 68;               // padded row stride (floats) of the fp32 64x64 tiles
+constexpr uint32_t X_GEXACT = 50176;  // exact Gram only: f32 [65][kLdG] cumulative log-decay
+constexpr int kLdG = 129;             // its padded row stride (floats)
+// A sub-chunk log-decay sum below this sends its item to the exact Gram
+// (e^{64} leaves e^{24} of headroom below the fp32/bf16 maximum for q, k).
+constexpr float kExactBound = -64.f;
 constexpr uint32_t X_NAE = 32768;     // 17 KB f32 [64][LDN]  (N = tril(A_e) diag(beta))
 constexpr uint32_t X_TINVF = 50176;   // 17 KB f32 [64][LDN]  (T^{-1}); both dead after step 6
 constexpr uint32_t X_Y = 69632;       // while T^{-1} is built: K-major [n][t]
@@ -355,6 +360,109 @@ __device__ __forceinline__ void named_bar_sync(int id, int threads) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// ---- exact Gram of one per-channel item (step 2a), all 512 threads ----
+// Every pair factor is formed directly from the in-chunk cumulative
+// log-decay G as one exp of a difference <= 0, in fp32 on the CUDA cores, so
+// nothing overflows whatever g is; the results go into the same images
+// (A_w beta, B_w beta, B_e beta in bf16, N = A_e beta in fp32) as the Gram
+// readback.  Reads the raw q, k and g tiles and the decay step's sub-chunk
+// and half-sub-chunk sums; ends with a block barrier after its last write.
+// Kept out of line: only items with a steep sub-chunk run it.
+template <bool DECAY_FIRST>
+__device__ __noinline__ void exact_gram(unsigned char *sm, int L) {
+  const int tid = threadIdx.x, bI = tid >> 7, rh = (tid >> 6) & 1, c2 = (tid & 63) * 2;
+  unsigned char *sX = sm + OFF_X;
+  const unsigned char *sQ = sm + OFF_Q, *sK = sm + OFF_K;
+  const float *sG = reinterpret_cast<const float *>(sm + OFF_G);
+  const float *sGsum = reinterpret_cast<const float *>(sm + OFF_MISC + MISC_GSUM);
+  const float *sBeta = reinterpret_cast<const float *>(sm + OFF_MISC + MISC_BETA);
+  float *Gt = reinterpret_cast<float *>(sX + X_GEXACT);  // Gt[t + 1][c] = G_t, Gt[0][c] = 0
+  {
+    const float *xs = reinterpret_cast<const float *>(sm + OFF_MISC + MISC_XS);
+    float b0 = rh ? xs[(2 * bI) * DK + c2] : 0.f, b1 = rh ? xs[(2 * bI) * DK + c2 + 1] : 0.f;
+    for (int J = 0; J < bI; ++J) {
+      b0 += sGsum[J * DK + c2];
+      b1 += sGsum[J * DK + c2 + 1];
+    }
+    if (bI == 0 && rh == 0) Gt[c2] = Gt[c2 + 1] = 0.f;
+#pragma unroll
+    for (int r = 0; r < 8; ++r) {
+      const int t = 16 * bI + 8 * rh + r;
+      if (t < L) {
+        const float2 gg = *reinterpret_cast<const float2 *>(sG + t * DK + c2);
+        b0 += gg.x;
+        b1 += gg.y;
+      }
+      Gt[(t + 1) * kLdG + c2] = b0;
+      Gt[(t + 1) * kLdG + c2 + 1] = b1;
+    }
+  }
+  __syncthreads();
+  // thread (row, chunk of 8 keys): key row i = row against keys j < i (A_w,
+  // A_e), query row t = row against keys j <= t (B_w, B_e)
+  const int row = tid >> 3, j0 = 8 * (tid & 7);
+  float aw[8], ae[8], bw[8], be[8];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) aw[u] = ae[u] = bw[u] = be[u] = 0.f;
+  if (j0 <= row && row < L) {
+    // keys in two halves of four (fewer live accumulators per channel loop)
+#pragma unroll
+    for (int hv = 0; hv < 2; ++hv) {
+#pragma unroll 1
+      for (int c = 0; c < DK; ++c) {
+        const uint32_t cb = (uint32_t)(c >> 6) * 8192;
+        const float Gi = Gt[(row + 1) * kLdG + c], Gpi = Gt[row * kLdG + c];
+        const float qv = ld_bf16(sQ, cb + kmajor_off(row, c & 63));
+        const float kv = ld_bf16(sK, cb + kmajor_off(row, c & 63));
+        const float arow = __expf(Gi - Gpi);  // a of the row's own token
+#pragma unroll
+        for (int u = 4 * hv; u < 4 * hv + 4; ++u) {
+          const int j = j0 + u;
+          if (j > row) continue;
+          const float Gj = Gt[(j + 1) * kLdG + c], Gpj = Gt[j * kLdG + c];
+          const float kj = ld_bf16(sK, cb + kmajor_off(j, c & 63));
+          const float qk = qv * kj, kk = kv * kj;
+          if (j == row) {  // the query's own key: e^{G_t - G_t} = 1, e^{G_t - Gp_t} = a_t
+            bw[u] += qk;
+            be[u] = fmaf(qk, DECAY_FIRST ? 1.f : arow, be[u]);
+          } else {
+            // K row: e^{Gp_i - G_j} (<= 1 for j < i); the rest follow by
+            // multiplying with a_i, a_j <= 1
+            const float faw = __expf((DECAY_FIRST ? Gi : Gpi) - Gj);
+            const float aj = DECAY_FIRST ? 1.f : __expf(Gj - Gpj);
+            const float fbw = DECAY_FIRST ? faw : faw * arow;  // e^{G_i - G_j}
+            aw[u] = fmaf(kk, faw, aw[u]);
+            ae[u] = fmaf(kk, faw * aj, ae[u]);
+            bw[u] = fmaf(qk, fbw, bw[u]);
+            be[u] = fmaf(qk, fbw * aj, be[u]);
+          }
+        }
+      }
+    }
+  }
+  __syncthreads();  // every read of the tables and tiles is done
+  {
+    float xw[8], xb[8], xe[8], xn[8];
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int j = j0 + u;
+      const float bj = sBeta[j];  // 0 past the chunk's length
+      const bool key = row < L && j < row, qry = row < L && j <= row;
+      xw[u] = key ? aw[u] * bj : 0.f;
+      xn[u] = key ? ae[u] * bj : 0.f;
+      xb[u] = qry ? bw[u] * bj : 0.f;
+      xe[u] = qry ? be[u] * bj : 0.f;
+    }
+    float *nae = reinterpret_cast<float *>(sX + X_NAE);
+    st16(sX + X_AWBW + kmajor_off(row, j0), pack8(xw));
+    st16(sX + X_AWBW + kmajor_off(64 + row, j0), pack8(xb));
+    st16(sX + X_BE + kmajor_off(row, j0), pack8(xe));
+    *reinterpret_cast<float4 *>(nae + row * LDN + j0) = make_float4(xn[0], xn[1], xn[2], xn[3]);
+    *reinterpret_cast<float4 *>(nae + row * LDN + j0 + 4) = make_float4(xn[4], xn[5], xn[6], xn[7]);
+  }
+  __syncthreads();
+}
+
 template <bool CHANNEL, bool DECAY_FIRST>
 __global__ void __launch_bounds__(kPrepThreads, 1)
 chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
@@ -389,6 +497,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   uint64_t *bar_oq = bar_tma + 4;    // the second O_intra term and Qc (one commit)
   uint64_t *bar_drain = bar_tma + 6;  // after an expired wait: every issuing thread's last MMAs
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + MISC_TSLOT);
+  volatile uint32_t *s_exact = reinterpret_cast<volatile uint32_t *>(sm + OFF_MISC + MISC_TSLOT + 4);
+  volatile uint32_t *s_fail = reinterpret_cast<volatile uint32_t *>(sm + OFF_MISC + MISC_BAR + 56);
 
   if (hdr[0] != KDA_DEVICE_OK) return;
   // persistent: this CTA walks (chunk, v-head) work items blockIdx.x,
@@ -410,6 +520,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mbar_init(bar_px, 1);
     mbar_init(bar_oq, 1);
     mbar_init(bar_drain, 4);
+    *s_exact = 0u;
+    s_fail[0] = s_fail[1] = 0u;
     mbar_fence_init();
   }
   tc_fence_before();
@@ -495,12 +607,20 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   if (tid < C) load_beta(work, ce, nbeta, ngsc);
 
-  // Every bounded wait below ANDs its verdict into `ok`; the block barriers
-  // after the waits take one CTA-wide verdict, and on a failure every thread
-  // leaves the work loop together (the status word already holds
-  // KDA_DEVICE_TIMEOUT), so an expired wait costs one bound, not one per item.
-  bool ok = true, aborted = false;
+  // A bounded wait that expires (the status word then holds
+  // KDA_DEVICE_TIMEOUT) raises the item's failure flag; at the top of the
+  // next item all threads take one verdict and leave the work loop together,
+  // so an expired wait costs at most one bound per wait site of one item,
+  // not one per item.  (Skipping a thread's later waits once one expired
+  // measured 8 % slower on the scalar-gate path.)
+  bool failed = false, aborted = false;
   int it = 0;
+  auto wait_bar = [&](uint64_t *bar, uint32_t parity, int32_t *err, int32_t code) {
+    if (!mbar_wait(bar, parity, err, code)) {
+      failed = true;
+      s_fail[it & 1] = 1u;
+    }
+  };
   for (; work < total; ++it, work += gridDim.x) {
   const int chunk = work / H_v, h = work - chunk * H_v;
   const int L = ce.len;
@@ -515,11 +635,19 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     if (next < total) load_beta(next, ce_next, nbeta, ngsc);
   }
   {
-    const bool landed = mbar_wait(bar_tma, it & 1, hdr, KDA_DEVICE_TIMEOUT);
-    ok &= landed;
-    if (landed) tma_done = it + 1;
+    wait_bar(bar_tma, it & 1, hdr, KDA_DEVICE_TIMEOUT);
+    if (!failed) tma_done = it + 1;
   }
-  if (__syncthreads_or(!ok)) { aborted = true; break; }
+  // One CTA-wide verdict per item: a wait that expired anywhere in the
+  // previous item ends the work loop on every thread.  Item i's waits raise
+  // flag i & 1, read by all threads after the next item's first barrier and
+  // cleared by thread 0 after a later barrier of that item, before any wait
+  // of item i + 2 can raise it again.
+  __syncthreads();
+  if (s_fail[(it + 1) & 1]) {
+    aborted = true;
+    break;
+  }
   // readbacks: warp (quad, qtr) reads TMEM lanes 32*quad .. +31, column quarter qtr
   const int quad = warp & 3, qtr = warp >> 2;
   const int lane_row = 32 * quad + lane;
@@ -579,13 +707,30 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       sGsum[bI * DK + c2] = s0 + os0;
       sGsum[bI * DK + c2 + 1] = s1 + os1;
     }
+    // The two-anchor Gram scales operands by up to 1/PB (PB: a channel's decay
+    // product over one 16-token sub-chunk).  A sub-chunk whose log-decay sum
+    // is below kExactBound would push them past the fp32/bf16 range: such an
+    // item takes the exact Gram below instead.
+    const bool steep = rh == 0 && (s0 + os0 < kExactBound || s1 + os1 < kExactBound);
+    if (__any_sync(0xffffffffu, steep) && lane == 0) *s_exact = 1u;  // every writer writes 1
   }
   // the previous item's image copies must have read the X region before it is rebuilt
   if (tid == kIoThread) bulk_wait_read0();
   __syncthreads();  // g is consumed: the next item's lands there
-  if (tid == kIoThread && next < total) {
+  const bool exact = *s_exact != 0;  // CTA-uniform; reset after the operand pass
+  if (tid == kIoThread && next < total && !exact) {
     load_g(next, ce_next);
     if (next + (int)gridDim.x < total) prefetch_l2(next + gridDim.x, ce_next2);
+  }
+
+  // ---- 2a. exact Gram (items with a steep sub-chunk only; slower than the
+  //          tensor-core Gram: ~2 exps per key pair and channel) ----
+  if (exact) {
+    exact_gram<DECAY_FIRST>(sm, L);
+    if (tid == kIoThread && next < total) {  // g is consumed
+      load_g(next, ce_next);
+      if (next + (int)gridDim.x < total) prefetch_l2(next + gridDim.x, ce_next2);
+    }
   }
 
   // ---- 3. one pass builds every operand of the chunk ----
@@ -668,15 +813,17 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float2 kw = __fmul2_rn(k, rw), ke = __fmul2_rn(k, re);
       const float2 kb = __fmul2_rn(k, bk), qb = __fmul2_rn(q, bq);
       const uint32_t rowK = (uint32_t)(32 * bI + 8 * rh + r) * 128 + x, rowQ = rowK + 16 * 128;
-      // Gram right operand (keys scaled to their group's anchor)
-      st4(rbase + rowK, __fmul2_rn(kw, rf));
-      st4(rbase + rowQ, __fmul2_rn(ke, rf));
-      // Gram left operands: anchor E_0 (all rows), anchor E_2 (sub-chunks 2, 3)
-      st4(lbase + rowK, __fmul2_rn(kb, fa));
-      st4(lbase + rowQ, __fmul2_rn(qb, fa));
-      if (bI >= 2) {
-        st4(lbase + LEFT_G1 + rowK, __fmul2_rn(kb, fb));
-        st4(lbase + LEFT_G1 + rowQ, __fmul2_rn(qb, fb));
+      if (!exact) {  // the exact Gram's images occupy this region
+        // Gram right operand (keys scaled to their group's anchor)
+        st4(rbase + rowK, __fmul2_rn(kw, rf));
+        st4(rbase + rowQ, __fmul2_rn(ke, rf));
+        // Gram left operands: anchor E_0 (all rows), anchor E_2 (sub-chunks 2, 3)
+        st4(lbase + rowK, __fmul2_rn(kb, fa));
+        st4(lbase + rowQ, __fmul2_rn(qb, fa));
+        if (bI >= 2) {
+          st4(lbase + LEFT_G1 + rowK, __fmul2_rn(kb, fb));
+          st4(lbase + LEFT_G1 + rowQ, __fmul2_rn(qb, fb));
+        }
       }
       // K e^{Gp} over k, q e^{G} over q (same element, same owner), beta K e^{G_L - G|Gp}
       st4(kbase + koff, __fmul2_rn(kb, ei));
@@ -693,7 +840,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   // ---- 4. Gram MMAs: per anchor group A, [K;Q] rows x 64 key columns (w, e of
   //         two key sub-chunks); one issuing thread per group ----
-  if (tid == 0 || tid == 32) {
+  if (tid == 0) *s_exact = 0u;  // every thread holds its copy of the flag
+  if ((tid == 0 || tid == 32) && exact) {
+    mbar_arrive(bar_mma);  // the phase completes with no product: the exact Gram is written
+  } else if (tid == 0 || tid == 32) {
     const int A = tid >> 5;
     constexpr uint32_t ID = idesc_bf16(128, 64, false, false);
     const uint32_t a_base = smem_u32(sX + X_LEFT + A * LEFT_G1);
@@ -705,7 +855,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mma_commit(bar_mma);
   }
   __syncwarp();
-  ok &= mbar_wait(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);
+  wait_bar(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
 
   // ---- 5. Gram readback: masked, beta-scaled, into the next operands ----
@@ -713,7 +863,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // sub-chunk J.  Blocks with J > I are zero; inside J == I the strict (keys) or
   // inclusive (queries) lower triangle survives.  Rows and keys past the chunk's
   // length are zero already (k = q = beta = 0 there).
-  {
+  if (!exact) {
     const int I = quad, J = qtr, s = lane;
     const bool isK = s < 16;
     const int i = 16 * I + (s & 15);
@@ -765,7 +915,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   }
   fence_async_smem();  // the images are operands of the next products
-  if (__syncthreads_or(!ok)) { aborted = true; break; }
+  __syncthreads();
   } else {
   // ---- 2'. scalar gate: every decay factor is a per-token scalar, so the Gram
   //          products take the raw tiles and the factors are applied to the
@@ -891,7 +1041,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   }
   __syncwarp();
-  ok &= mbar_wait(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);
+  wait_bar(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
 
   // ---- 5'. Gram readback: TMEM lane r < 64 is key row i = r, lane 64 + t query
@@ -979,11 +1129,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   }
   fence_async_smem();  // the images are operands of the next products
-  if (__syncthreads_or(!ok)) { aborted = true; break; }
+  __syncthreads();
   // the raw q, k tiles are consumed (Gram and image pass): the next item's load now
   if (tid == kIoThread && next < total) load_qk(next, ce_next, false);
   }  // scalar gate
 
+  if (tid == 0) s_fail[(it + 1) & 1] = 0u;  // the previous item's flag, read by now
   // ---- 6. products that need no T^{-1}, issued before it is built:
   //         Y^T = V^T (A_w beta)^T;  O_intra = tril(B_w) beta V (rows t < 64 of an
   //         M = 128 product whose upper 64 rows read the bytes after the operand
@@ -1091,7 +1242,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     }
   } else {
     // warps 8-15, meanwhile: Y (lanes n, cols i) -> K-major [n][t]
-    ok &= mbar_wait(bar_yo, it & 1, hdr, KDA_DEVICE_TIMEOUT);
+    wait_bar(bar_yo, it & 1, hdr, KDA_DEVICE_TIMEOUT);
     // the step-6 products were the last to read v: the next item's v tile now
     if (tid == kIoThread && next < total) load_v(next, ce_next, !CHANNEL);
     tc_fence_after();
@@ -1109,7 +1260,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   fence_async_smem();
   tc_fence_before();
-  if (__syncthreads_or(!ok)) { aborted = true; break; }
+  __syncthreads();
   tc_fence_after();
 
   // ---- 8. W^T = (K e^{Gp})^T T^{-T};  U^T = Y^T T^{-T} ----
@@ -1129,7 +1280,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mma_commit(bar_mma);
   }
   __syncwarp();
-  ok &= mbar_wait(bar_mma, 1, hdr, KDA_DEVICE_TIMEOUT);
+  wait_bar(bar_mma, 1, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
   {
     // W (lanes c, cols t) -> K-major [c][t]; U (lanes n, cols t) -> K-major [n][t]
@@ -1151,7 +1302,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   fence_async_smem();
   tc_fence_before();
-  if (__syncthreads_or(!ok)) { aborted = true; break; }
+  __syncthreads();
   tc_fence_after();
 
   // ---- 9. thread 32: K_b^T beta W (for P), X = W^T (B_e beta)^T (for Q');
@@ -1183,7 +1334,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     mma_commit(bar_oq);
   }
   __syncwarp();
-  ok &= mbar_wait(bar_px, it & 1, hdr, KDA_DEVICE_TIMEOUT);
+  wait_bar(bar_px, it & 1, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
   // P and Q' leave TMEM for the slot while the last products run (disjoint columns)
   {
@@ -1221,7 +1372,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   fence_async_smem();
   tc_fence_before();
-  if (__syncthreads_or(!ok)) { aborted = true; break; }  // the P / Q' images are written
+  __syncthreads();  // the P / Q' images are written
   tc_fence_after();
   if (tid == kIoThread) {  // P and Q' images -> workspace slot
     bulk_s2g(slot + SLOT_P, sX + X_PI, 32768);
@@ -1229,7 +1380,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     bulk_commit();
     if (CHANNEL && next < total) load_qk(next, ce_next, true);  // Q' has read the q tile
   }
-  ok &= mbar_wait(bar_oq, it & 1, hdr, KDA_DEVICE_TIMEOUT);
+  wait_bar(bar_oq, it & 1, hdr, KDA_DEVICE_TIMEOUT);
   tc_fence_after();
   {
     // warp (quad, qtr) holds rows 32 quad + lane, value columns 32 qtr .. +31,
@@ -1258,7 +1409,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   fence_async_smem();
   tc_fence_before();
-  if (__syncthreads_or(!ok)) { aborted = true; break; }
+  __syncthreads();
   tc_fence_after();
   if (tid == kIoThread) {  // Qc and O_intra images -> workspace slot
     bulk_s2g(slot + SLOT_QC, sX + X_QCI, 32768);
@@ -1269,6 +1420,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   ce_next = ce_next2;
   }  // work items
 
+  // a wait in the last item may have expired after the final verdict
+  aborted = __syncthreads_or(aborted || failed) != 0;
   if (aborted) {
     // Nothing may still write this CTA's shared memory or TMEM when it exits:
     // the issuing threads' last products finish (a commit arrives once every

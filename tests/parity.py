@@ -141,7 +141,7 @@ def prefill_device_inputs(x, device="cuda"):
     return d
 
 
-def oracle_prefill(x, heads=None, threads=None):
+def oracle_prefill(x, heads=None, threads=None, order="erase_then_decay"):
     """Run the oracle on a PrefillInputs (optionally only the v-heads in ``heads``,
     each given its own copy of its q/k head).  Returns (o [Ttot, nh, d_v],
     final [N, nh, d_k, d_v])."""
@@ -150,9 +150,10 @@ def oracle_prefill(x, heads=None, threads=None):
     s0 = x.initial_state
     if heads is None:
         return oracle.gated_delta(x.q32, x.k32, x.v32, x.g, x.beta, s0,
-                                  x.cu_seqlens.astype(np.int64), threads=threads)
+                                  x.cu_seqlens.astype(np.int64), threads=threads, order=order)
     group = w.H_v // w.H_qk
     hk = [h // group for h in heads]
     return oracle.gated_delta(
         x.q32[:, hk], x.k32[:, hk], x.v32[:, heads], x.g[:, heads], x.beta[:, heads],
-        None if s0 is None else s0[:, heads], x.cu_seqlens.astype(np.int64), threads=threads)
+        None if s0 is None else s0[:, heads], x.cu_seqlens.astype(np.int64), threads=threads,
+        order=order)

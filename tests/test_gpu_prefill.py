@@ -46,9 +46,9 @@ def _run(x, **kw):
     return o, sT.cpu().numpy()
 
 
-def _check(x, heads=None, tol=None, regress=None):
-    o, sT = _run(x)
-    ro, rs = oracle_prefill(x, heads)
+def _check(x, heads=None, tol=None, regress=None, **kw):
+    o, sT = _run(x, **kw)
+    ro, rs = oracle_prefill(x, heads, **kw)
     if heads is not None:
         o, sT = o[:, heads], sT[:, heads]
     tol = tol or tol_for(x.w.io_dtype)
@@ -105,6 +105,28 @@ def test_strong_decay(gate, scale):
     w = W.WORKLOADS[base].replace(T=200, H_qk=2, H_v=2 if gate == "channel" else 4,
                                   gate_scale=scale, init_state=True)
     _check(W.make_prefill(w, seed=13))
+
+
+@pytest.mark.parametrize("scale,order", [(4.0, "erase_then_decay"), (8.0, "erase_then_decay"),
+                                         (4.0, "decay_then_erase")])
+def test_kda_steep_decays(scale, order):
+    """Per-token log-decays down to -16 and beyond on the bf16 tensor-core
+    path.  A 16-token sub-chunk whose log-decay sum (for some channel) falls
+    below -64 would push the two-anchor Gram's scale factors past the
+    fp32/bf16 range; the kernel computes such items' Grams exactly instead.
+    At scale 4 both kinds of item occur (the ragged last chunk is not steep),
+    at scale 8 (mean -6.5 per token) every full chunk takes the exact Gram."""
+    w = W.WORKLOADS["kda_prefill"].replace(T=200, H_qk=2, H_v=2, gate_scale=scale,
+                                           init_state=True)
+    x = W.make_prefill(w, seed=17)
+    assert x.g.min() <= -15.0
+    # sub-chunk sums of the log-decay per (16-token sub-chunk, head, channel)
+    gp = np.zeros((256,) + x.g.shape[1:], np.float64)
+    gp[:200] = x.g
+    sums = gp.reshape(16, 16, *x.g.shape[1:]).sum(axis=1)
+    steep = (sums < -64.0).any(axis=(-1,)).reshape(4, 4, -1).any(axis=1)  # per (chunk, head)
+    assert steep.any() and (scale > 4 or not steep.all())
+    _check(x, order=order)
 
 
 def test_gdn_unshared_heads():
