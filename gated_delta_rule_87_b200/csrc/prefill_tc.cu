@@ -1476,9 +1476,9 @@ struct ScanCfg {
   static constexpr uint32_t TD_S = 0, TD_O = NS;          // TMEM columns: (P S), (Q' S) x 2
   static constexpr uint32_t TMEM_COLS = NS == 32 ? 128 : 256;
 };
-constexpr int kScanThreads = 288;
-constexpr int kScanMmaWarp = 6, kScanLoadWarp = 7, kScanOutMmaWarp = 8;
-constexpr uint32_t kScanEmptyCount = 128 + 64 + 2;  // chain + output threads + two MMA commits
+constexpr int kScanThreads = 256;
+constexpr int kScanMmaWarp = 6, kScanLoadWarp = 7;
+constexpr uint32_t kScanEmptyCount = 128 + 64 + 1;  // chain + output threads + MMA commit
 
 // byte offset of the 16-byte chunk `ch` of state-operand row c (MN-major, NS columns)
 template <int NS>
@@ -1506,8 +1506,7 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
   uint64_t *ds_full = sb_ready + 2;   // (P S) done (commit)
   uint64_t *do_full = ds_full + 1;    // [2] (Q' S) done (commit)
   uint64_t *do_free = do_full + 2;    // [2] (Q' S) read (output)
-  uint64_t *drain = do_free + 2;      // [2] final commits of the two MMA warps
-  uint64_t *ds_done = drain + 2;      // [2] (P S) of chunk u done, for the output issue (u & 1)
+  uint64_t *drain = do_free + 2;      // final commit of the MMA warp
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + Cfg::OFF_MISC + 192);
 
   if (hdr[0] != KDA_DEVICE_OK) return;
@@ -1532,10 +1531,7 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
       mbar_init(&do_free[b], 64);
     }
     mbar_init(ds_full, 1);
-    mbar_init(&drain[0], 1);
-    mbar_init(&drain[1], 1);
-    mbar_init(&ds_done[0], 1);
-    mbar_init(&ds_done[1], 1);
+    mbar_init(drain, 1);
     mbar_fence_init();
   }
   tc_fence_before();
@@ -1583,58 +1579,47 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
       for (int u = (issued > S ? issued - S : 0); u < issued; ++u)
         mbar_wait(&full[u % S], (u / S) & 1, err, KDA_DEVICE_TIMEOUT);
     }
-  } else if (warp == kScanMmaWarp || warp == kScanOutMmaWarp) {
+  } else if (warp == kScanMmaWarp) {
     // ---------------- tensor-core issue ----------------
-    // Two issuing warps, so that neither product waits for the other's
-    // issue (one thread issues a tcgen05.mma every ~60 cycles): warp 6 the
-    // chain product P S of each chunk as soon as S_u is written, warp 8 the
-    // output product Q' S once the chain product has landed (it then runs in
-    // the tensor pipe while the chain warps update the state).  Each warp
-    // runs its loop converged and computes the descriptors (warp-uniform
-    // values); one elected lane issues.
-    const bool chain_warp = warp == kScanMmaWarp;
+    // The whole warp runs the loop and computes the operand descriptors
+    // (warp-uniform values); one elected lane issues the products.
     constexpr uint32_t idS = idesc_bf16(128, NS, false, true);  // P K-major, S MN-major
     constexpr uint32_t idO = idesc_bf16(128, NS, true, true);   // Q' MN-major, S MN-major
     for (int u = 0; u < nch; ++u) {
       const int st = u % S, b = u & 1;
       if (!mbar_wait_warp(&full[st], (u / S) & 1, err, KDA_DEVICE_TIMEOUT)) break;
       if (!mbar_wait_warp(&sb_ready[b], (u >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
-      if (!chain_warp) {
-        // (a barrier per chunk parity: the chain can be one product ahead)
-        if (!mbar_wait_warp(&ds_done[b], (u >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
-        if (u >= 2 && !mbar_wait_warp(&do_free[b], ((u - 2) >> 1) & 1, err, KDA_DEVICE_TIMEOUT))
-          break;
-      }
       tc_fence_after();
       const uint32_t stage = smem_u32(sm + st * Cfg::ST_BYTES);
       const uint32_t sb = smem_u32(sm + Cfg::OFF_SB + b * Cfg::SB_BYTES);
       uint64_t da[8], dbs[8];
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk) {
-        da[kk] = chain_warp ? desc_kmajor(stage + Cfg::ST_P, 16 * kk, 16384)
-                            : desc_mnmajor(stage + Cfg::ST_QP, 16 * kk, 16384);
+        da[kk] = desc_kmajor(stage + Cfg::ST_P, 16 * kk, 16384);
         dbs[kk] = sop_desc<NS>(sb, kk);
       }
       if (elect_one()) {
-        if (chain_warp) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) mma_bf16(tm + Cfg::TD_S, da[kk], dbs[kk], idS, kk > 0);
-          mma_commit(ds_full);
-          mma_commit(&ds_done[b]);
-        } else {
+        for (int kk = 0; kk < 8; ++kk) mma_bf16(tm + Cfg::TD_S, da[kk], dbs[kk], idS, kk > 0);
+        mma_commit(ds_full);
+      }
+      __syncwarp();
+      if (u >= 2 && !mbar_wait_warp(&do_free[b], ((u - 2) >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
+      tc_fence_after();
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk)
-            mma_bf16(tm + Cfg::TD_O + NS * b, da[kk], dbs[kk], idO, kk > 0);
-          mma_commit(&do_full[b]);
-        }
+      for (int kk = 0; kk < 8; ++kk) da[kk] = desc_mnmajor(stage + Cfg::ST_QP, 16 * kk, 16384);
+      if (elect_one()) {
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk) mma_bf16(tm + Cfg::TD_O + NS * b, da[kk], dbs[kk], idO, kk > 0);
+        mma_commit(&do_full[b]);
         mma_commit(&empty[st]);
       }
       __syncwarp();
     }
     // every issued product has finished before TMEM is released
-    if (elect_one()) mma_commit(&drain[chain_warp ? 0 : 1]);
+    if (elect_one()) mma_commit(drain);
     __syncwarp();
-    mbar_wait_warp(&drain[chain_warp ? 0 : 1], 0, err, KDA_DEVICE_TIMEOUT);
+    mbar_wait_warp(drain, 0, err, KDA_DEVICE_TIMEOUT);
   } else if (warp < 4) {
     // ---------------- the state chain: row i, NS columns ----------------
     const int i = 32 * warp + lane;
@@ -1693,10 +1678,6 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
         }
       }
       if (u + 1 < nch) {
-        // S_{u+1} replaces S_{u-1}, which the output product of chunk u - 1
-        // (the other issuing warp) reads: it has landed
-        if (u >= 1 && !mbar_wait(&do_full[(u - 1) & 1], ((u - 1) >> 1) & 1, err, KDA_DEVICE_TIMEOUT))
-          break;
         write_operand((u + 1) & 1);
         mbar_arrive(&sb_ready[(u + 1) & 1]);
       }
