@@ -56,9 +56,13 @@ def test_noalloc_matches_workspace_entry_point_twice():
 def test_noalloc_rejects_problems_beyond_its_scratch():
     import gated_delta_rule_87_b200 as gdr
     L = gdr.lib()
-    # T = 4096, H = 32 needs about 200 MB of scratch: far above 64 MiB.
-    fake = 1 << 16  # never dereferenced: the size check comes first
+    # 128 sequences x 32 heads: a 32 KB state image per chain alone is 128 MiB.
+    # The size is checked here first: the call below passes unmapped pointers
+    # and must never get past the library's host-side size check.
+    B, T, H = 128, 64, 32
+    assert L.kda_chunk_fwd_workspace_size(B, T, H, 128, 128, 0, 1) > (64 << 20)
+    fake = 1 << 16
     st = L.kda_chunk_fwd_noalloc(fake, fake, fake, fake, fake, fake * 2, None, None, None, 0,
-                                 1, 4096, 32, 128, 128, 1, None)
+                                 B, T, H, 128, 128, 1, None)
     assert st == gdr.KDA_ERR_WORKSPACE
     assert b"64" in L.kda_last_error() or b"67108864" in L.kda_last_error()
