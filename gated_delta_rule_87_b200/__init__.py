@@ -14,6 +14,7 @@ one table", rows "KDA" and "Gated DeltaNet"; column-vector keys):
 """
 from __future__ import annotations
 
+import contextlib
 import ctypes
 import os
 import threading
@@ -23,6 +24,7 @@ __all__ = [
     "lib", "library_path", "KdaError", "kda_chunk_fwd", "gdn_chunk_fwd", "kda_decode_step",
     "gdn_decode_step", "kda_recurrent_fwd", "gdn_recurrent_fwd", "state_gather", "state_scatter",
     "chunk_workspace_size", "check_device_status", "EXPORTED_SYMBOLS",
+    "checked_library_path", "use_library", "bounds_checked", "bounds_violations",
     "trace_enable", "trace_read", "ERASE_THEN_DECAY", "DECAY_THEN_ERASE",
     "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
     "KDA_ERR_DEVICE_CHECK", "KDA_ERR_WORKSPACE",
@@ -30,6 +32,8 @@ __all__ = [
 
 _PKG = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_PKG, "libgated_delta.so")
+# the bounds-checked build of the same sources (see kda_bounds_checked)
+checked_library_path = os.path.join(_PKG, "libgated_delta_checked.so")
 
 KDA_OK, KDA_ERR_INVALID_ARG, KDA_ERR_UNSUPPORTED, KDA_ERR_CUDA, KDA_ERR_DEVICE_CHECK, \
     KDA_ERR_WORKSPACE = range(6)
@@ -46,7 +50,8 @@ EXPORTED_SYMBOLS = (
     "kda_check_device_status", "kda_status_string", "kda_last_error", "kda_abi_version",
     "kda_trace_enable", "kda_trace_read", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_ex",
     "gdn_chunk_fwd_ex", "kda_recurrent_fwd", "gdn_recurrent_fwd", "kda_state_gather",
-    "kda_state_scatter", "kda_selftest_wait_timeout",
+    "kda_state_scatter", "kda_selftest_wait_timeout", "kda_bounds_checked",
+    "kda_bounds_violations",
 )
 
 _lock = threading.Lock()
@@ -75,6 +80,8 @@ _SIGS = {
     "kda_trace_enable": ([_i32], ctypes.c_int),
     "kda_chunk_fwd_noalloc": ([_vp] * 9 + [_i32] * 6 + [ctypes.c_int, _vp], ctypes.c_int),
     "kda_trace_read": ([ctypes.c_char_p, _i32, ctypes.POINTER(ctypes.c_float), _i32], _i32),
+    "kda_bounds_checked": ([], _i32),
+    "kda_bounds_violations": ([_vp, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
 }
 
 
@@ -84,22 +91,63 @@ class KdaError(RuntimeError):
         super().__init__(f"{detail} (status {status})")
 
 
-def lib() -> ctypes.CDLL:
-    """Load ``libgated_delta.so`` (raises if it has not been built)."""
-    global _lib
+_libs = {}                   # path -> loaded CDLL
+_active_path = library_path  # the library the calls below go through
+
+
+def _load(path: str) -> ctypes.CDLL:
     with _lock:
-        if _lib is None:
-            if not os.path.exists(library_path):
+        L = _libs.get(path)
+        if L is None:
+            if not os.path.exists(path):
                 raise ImportError(
-                    f"{library_path} is missing: build it with "
+                    f"{path} is missing: build it with "
                     "`python -m gated_delta_rule_87_b200.build` (nvcc, sm_100a)")
-            L = ctypes.CDLL(library_path)
+            L = ctypes.CDLL(path)
             for name, (args, res) in _SIGS.items():
                 f = getattr(L, name)
                 f.argtypes = args
                 f.restype = res
-            _lib = L
-    return _lib
+            _libs[path] = L
+    return L
+
+
+def lib() -> ctypes.CDLL:
+    """Load ``libgated_delta.so`` (raises if it has not been built), or the
+    library selected by :func:`use_library`."""
+    global _lib
+    L = _load(_active_path)
+    if _active_path == library_path:
+        _lib = L
+    return L
+
+
+@contextlib.contextmanager
+def use_library(path: str):
+    """Route every call of this module through the library at ``path`` (for
+    instance :data:`checked_library_path`) inside the ``with`` block."""
+    global _active_path
+    prev = _active_path
+    L = _load(path)
+    _active_path = path
+    try:
+        yield L
+    finally:
+        _active_path = prev
+
+
+def bounds_checked() -> bool:
+    """True when the active library is the bounds-checked build."""
+    return bool(lib().kda_bounds_checked())
+
+
+def bounds_violations() -> int:
+    """Waits for the current stream and returns the out-of-bounds accesses the
+    active library's kernels caught (and skipped) since the last call."""
+    n = ctypes.c_uint32(0)
+    _check(lib().kda_bounds_violations(_stream_handle(None, None), ctypes.byref(n)),
+           "kda_bounds_violations")
+    return int(n.value)
 
 
 def _check(status: int, what: str):

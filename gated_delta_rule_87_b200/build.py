@@ -1,6 +1,6 @@
 """Build the CUDA library ``libgated_delta.so`` in-tree (sm_100a).
 
-    python -m gated_delta_rule_87_b200.build [--force]
+    python -m gated_delta_rule_87_b200.build [--force] [--no-checked]
 
 nvcc cross-compiles for sm_100a without a GPU.  The library links the CUDA
 runtime statically and needs no libcuda at link time.
@@ -19,6 +19,9 @@ CSRC = os.path.join(PKG, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(PKG, "libgated_delta.so")
 BUILD_DIR = os.path.join(PKG, "_build")
+# the same sources with every kernel-computed global index checked (sanitizer substitute)
+LIB_CHECKED = os.path.join(PKG, "libgated_delta_checked.so")
+BUILD_DIR_CHECKED = os.path.join(PKG, "_build_checked")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 NVCC_FLAGS = ["-O3", "-std=c++17", "-lineinfo", 
@@ -49,16 +52,17 @@ def _stale(target, deps) -> bool:
     return any(os.path.getmtime(d) > t for d in deps)
 
 
-def build(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
-    os.makedirs(BUILD_DIR, exist_ok=True)
+def _build_variant(lib_path: str, build_dir: str, defines, force: bool, verbose: bool) -> str:
+    os.makedirs(build_dir, exist_ok=True)
     objs = []
     procs = []
     hdrs = headers()
     for src in sources():
-        obj = os.path.join(BUILD_DIR, os.path.basename(src).replace(".cu", ".o"))
+        obj = os.path.join(build_dir, os.path.basename(src).replace(".cu", ".o"))
         objs.append(obj)
         if force or _stale(obj, [src] + hdrs):
-            cmd = [nvcc(), *ARCH, *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-c", src, "-o", obj]
+            cmd = [nvcc(), *ARCH, *NVCC_FLAGS, *defines, "-I", INCLUDE, "-I", CSRC, "-c", src,
+                   "-o", obj]
             if verbose:
                 cmd += ["-Xptxas", "-v"]
             procs.append((src, subprocess.Popen(cmd, stdout=subprocess.PIPE,
@@ -72,14 +76,24 @@ def build(force: bool = False, verbose: bool = False, jobs: int = 0) -> str:
             failed.append(src)
     if failed:
         raise RuntimeError("nvcc failed for: " + ", ".join(os.path.basename(f) for f in failed))
-    if force or procs or _stale(LIB, objs):
-        tmp = LIB + f".tmp{os.getpid()}"
+    if force or procs or _stale(lib_path, objs):
+        tmp = lib_path + f".tmp{os.getpid()}"
         cmd = [nvcc(), *ARCH, "-shared", "-cudart", "static", "-o", tmp, *objs]
         subprocess.run(cmd, check=True)
-        os.replace(tmp, LIB)
+        os.replace(tmp, lib_path)
+    return lib_path
+
+
+def build(force: bool = False, verbose: bool = False, checked: bool = True) -> str:
+    """Build ``libgated_delta.so`` and (unless ``checked`` is False) the
+    bounds-checked ``libgated_delta_checked.so`` from the same sources."""
+    _build_variant(LIB, BUILD_DIR, [], force, verbose)
+    if checked:
+        _build_variant(LIB_CHECKED, BUILD_DIR_CHECKED, ["-DGDR_BOUNDS_CHECK"], force, verbose)
     return LIB
 
 
 if __name__ == "__main__":
-    build(force="--force" in sys.argv, verbose="-v" in sys.argv)
+    build(force="--force" in sys.argv, verbose="-v" in sys.argv,
+          checked="--no-checked" not in sys.argv)
     print(LIB)

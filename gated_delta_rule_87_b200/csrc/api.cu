@@ -141,6 +141,8 @@ __global__ void check_cu_seqlens_kernel(const int32_t *__restrict__ cu, int num_
   if (__syncthreads_or(bad) && threadIdx.x == 0) *status = KDA_DEVICE_BAD_CU_SEQLENS;
 }
 
+GDR_DEFINE_OOB_COUNTER(oob_count_api)
+
 cudaError_t launch_check_cu_seqlens(const int32_t *cu, int num_seqs, int T, int32_t *status,
                                     cudaStream_t stream) {
   check_cu_seqlens_kernel<<<1, 256, 0, stream>>>(cu, num_seqs, T, status);
@@ -382,6 +384,29 @@ kda_status_t kda_check_device_status(const void *workspace, void *stream, int32_
   if (device_code) *device_code = code;
   if (code != KDA_DEVICE_OK)
     return fail(KDA_ERR_DEVICE_CHECK, "device check failed with code %d", code);
+  return KDA_OK;
+}
+
+int32_t kda_bounds_checked(void) {
+#ifdef GDR_BOUNDS_CHECK
+  return 1;
+#else
+  return 0;
+#endif
+}
+
+kda_status_t kda_bounds_violations(void *stream, uint32_t *count) {
+  if (!count) return fail(KDA_ERR_INVALID_ARG, "count is NULL");
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess) return cuda_fail(e, "synchronising before reading the bounds counters");
+  const unsigned int parts[] = {gdr::oob_count_prefill_tc(), gdr::oob_count_prefill_simt(),
+                                gdr::oob_count_decode(), gdr::oob_count_api()};
+  uint64_t total = 0;
+  for (unsigned int p : parts) {
+    if (p == ~0u) return fail(KDA_ERR_CUDA, "a bounds counter could not be read");
+    total += p;
+  }
+  *count = total > 0xffffffffull ? 0xffffffffu : (uint32_t)total;
   return KDA_OK;
 }
 

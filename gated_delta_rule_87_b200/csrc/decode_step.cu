@@ -124,11 +124,15 @@ recurrent_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *_
   __shared__ __align__(16) BlockVecs<D_K, D_V, TB> bv;
   __shared__ __align__(16) float s_red[2][2][kWarps][D_V];  // [token parity][r | p][warp][column]
 
+  // extents of the token rows (the bounds-checked build compares against them)
+  const int64_t tokens = (int64_t)(gridDim.x / H_v) * T;
+  (void)tokens;
   const int64_t slot = slots ? (int64_t)__ldg(slots + n) : (int64_t)n;
   if (slot < 0 || slot >= num_slots) {  // padding entry: zero outputs, state untouched
     for (int e = threadIdx.x; e < T * D_V; e += kWarps * 32) {
       const int t = e / D_V, c = e - t * D_V;
-      io<IO>::store(o + (((size_t)n * T + t) * H_v + h) * D_V + c, 0.f);
+      if (GDR_IN_BOUNDS((int64_t)n * T + t < tokens))
+        io<IO>::store(o + (((size_t)n * T + t) * H_v + h) * D_V + c, 0.f);
     }
     return;
   }
@@ -144,7 +148,7 @@ recurrent_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *_
   // One warp stages token t into block entry tt: the row vectors, the value
   // and the readout coefficients (k.q and k.(a.q) by a warp reduction).
   auto stage = [&](int tt, int t) {
-    const size_t tok = token_base(t);
+    const size_t tok = GDR_IN_BOUNDS((int64_t)token_base(t) < tokens) ? token_base(t) : 0;
     const float b = __ldg(beta + tok * H_v + h);
     const float gsc = CHANNEL_GATE ? 0.f : __ldg(g + tok * H_v + h);
     float kq = 0.f, kaq = 0.f;
@@ -247,7 +251,7 @@ recurrent_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO *_
         ps += __shfl_xor_sync(0xffffffffu, ps, off);
         rs += __shfl_xor_sync(0xffffffffu, rs, off);
       }
-      if (opart == 0)
+      if (opart == 0 && GDR_IN_BOUNDS((int64_t)token_base(t0 + tt) < tokens))
         io<IO>::store(o + (token_base(t0 + tt) * H_v + h) * D_V + ocol,
                       ps - bv.coef[tt][0] * rs + bv.coef[tt][1] * bv.v[tt][ocol]);
     }
@@ -315,6 +319,8 @@ __global__ void state_copy_kernel(const float4 *__restrict__ src, const int32_t 
 }
 
 }  // namespace
+
+GDR_DEFINE_OOB_COUNTER(oob_count_decode)
 
 cudaError_t launch_recurrent(const DecodeArgs &a, cudaStream_t stream) {
   if (a.N == 0) return cudaSuccess;

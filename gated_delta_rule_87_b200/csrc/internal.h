@@ -29,6 +29,13 @@ void set_last_error(const char *msg);
 // Multiprocessor count of the current device.
 int sm_count();
 
+// Bounds-checked build: violations counted by each translation unit's
+// kernels since the last read (0 in the normal build; ~0u if unreadable).
+unsigned int oob_count_prefill_tc();
+unsigned int oob_count_prefill_simt();
+unsigned int oob_count_decode();
+unsigned int oob_count_api();
+
 // Token-by-token form: T tokens for each of N sequences ([N, T, H, d]
 // layout), state updated in place.  T = 1 is one decode step.
 struct DecodeArgs {

@@ -80,6 +80,10 @@ prefill_simt_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO
   const int tid = threadIdx.x;
   const int col0 = slice * NS;
 
+  // token rows of the whole batch (the bounds-checked build compares against it)
+  const int nseqs = (int)(gridDim.x / (NSLICE * H_v));
+  const int64_t T_total = cu ? (int64_t)cu[nseqs] : (int64_t)nseqs * T;
+  (void)T_total;
   int64_t bos, eos;
   if (cu) {
     bos = cu[n];
@@ -109,7 +113,7 @@ prefill_simt_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO
     for (int e = tid; e < C * D_K; e += kThreads) {
       const int t = e / D_K, c = e % D_K;
       float kk = 0.f, qq = 0.f, gg = 0.f;
-      if (t < L) {
+      if (t < L && GDR_IN_BOUNDS(c0 + t < T_total)) {
         const size_t off = ((size_t)(c0 + t) * H_qk + hk) * D_K + c;
         kk = io<IO>::load(k + off);
         qq = io<IO>::load(q + off);
@@ -122,9 +126,12 @@ prefill_simt_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO
     }
     for (int e = tid; e < C * NS; e += kThreads) {
       const int t = e / NS, j = e % NS;
-      sm.V[t][j] = (t < L) ? io<IO>::load(v + ((size_t)(c0 + t) * H_v + h) * D_V + col0 + j) : 0.f;
+      sm.V[t][j] = (t < L && GDR_IN_BOUNDS(c0 + t < T_total))
+                       ? io<IO>::load(v + ((size_t)(c0 + t) * H_v + h) * D_V + col0 + j) : 0.f;
     }
-    if (tid < C) sm.beta[tid] = (tid < L) ? __ldg(beta + (size_t)(c0 + tid) * H_v + h) : 0.f;
+    if (tid < C)
+      sm.beta[tid] = (tid < L && GDR_IN_BOUNDS(c0 + tid < T_total))
+                         ? __ldg(beta + (size_t)(c0 + tid) * H_v + h) : 0.f;
     __syncthreads();
 
     // 2. in-chunk cumulative sum of the log-decay, in token order
@@ -205,7 +212,7 @@ prefill_simt_kernel(const IO *__restrict__ q, const IO *__restrict__ k, const IO
     // 6. outputs o = (Q.e^{G}) S_0 + tril(B_w) beta V - tril(B_e) beta R
     for (int e = tid; e < C * NS; e += kThreads) {
       const int i = e / NS, j = e % NS;
-      if (i >= L) continue;
+      if (i >= L || !GDR_IN_BOUNDS(c0 + i < T_total)) continue;
       float acc = 0.f;
       for (int c = 0; c < D_K; ++c) acc = fmaf(sm.Q[i][c] * expf(sm.G[i][c]), sm.S[c][j], acc);
       for (int jj = 0; jj <= i; ++jj)
@@ -263,6 +270,8 @@ cudaError_t launch_io(const PrefillArgs &a, cudaStream_t s) {
 }
 
 }  // namespace
+
+GDR_DEFINE_OOB_COUNTER(oob_count_prefill_simt)
 
 cudaError_t launch_prefill_f32(const PrefillArgs &a, cudaStream_t stream) {
   if (a.bf16) {

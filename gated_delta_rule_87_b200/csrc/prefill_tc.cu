@@ -99,12 +99,13 @@ struct Chunks {
   const int32_t *seq_off, *order;
   int dense_T;  // > 0: dense batch of sequences of this length (no table)
   int per_seq;  // dense: chunks per sequence
+  int64_t T_total, max_chunks;  // extents of the token rows and of the chunk table / slots
   __device__ __forceinline__ ChunkEntry entry(int ck) const {
     if (dense_T > 0) {
       const int n = ck / per_seq, j = ck - n * per_seq;
       return ChunkEntry{n, n * dense_T + j * C, min(C, dense_T - j * C), 0};
     }
-    return tab[ck];
+    return GDR_IN_BOUNDS(ck >= 0 && ck < max_chunks) ? tab[ck] : ChunkEntry{0, 0, 0, 0};
   }
   __device__ __forceinline__ int first(int n) const { return dense_T > 0 ? n * per_seq : seq_off[n]; }
   __device__ __forceinline__ int seq(int r) const { return dense_T > 0 ? r : order[r]; }
@@ -183,7 +184,7 @@ plan_kernel(const int32_t *__restrict__ cu, int num_seqs, int T, int T_total, in
         e.start = bos + j * C;
         e.len = min(C, len - j * C);
         e.pad = 0;
-        tab[first + j] = e;
+        if (GDR_IN_BOUNDS(first + j < (int64_t)T_total / C + num_seqs)) tab[first + j] = e;
       }
     }
     __syncthreads();
@@ -594,8 +595,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // beta (and the scalar gate) of an item, one token per thread tid < C
   auto load_beta = [&](int w, const ChunkEntry &e, float &b, float &gs) {
     const int hh = w % H_v;
-    b = (tid < e.len) ? __ldg(beta + (size_t)(e.start + tid) * H_v + hh) : 0.f;
-    gs = (!CHANNEL && tid < e.len) ? __ldg(g_scalar + (size_t)(e.start + tid) * H_v + hh) : 0.f;
+    const bool in = tid < e.len && GDR_IN_BOUNDS((int64_t)e.start + tid < chunks.T_total);
+    b = in ? __ldg(beta + (size_t)(e.start + tid) * H_v + hh) : 0.f;
+    gs = (!CHANNEL && in) ? __ldg(g_scalar + (size_t)(e.start + tid) * H_v + hh) : 0.f;
   };
   float nbeta = 0.f, ngsc = 0.f;  // the coming item's, loaded one item ahead
   ChunkEntry ce = entry(work), ce_next = entry(work + gridDim.x);
@@ -1374,9 +1376,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   tc_fence_before();
   __syncthreads();  // the P / Q' images are written
   tc_fence_after();
-  if (tid == kIoThread) {  // P and Q' images -> workspace slot
+  const bool slot_ok = tid != kIoThread || GDR_IN_BOUNDS(chunk < chunks.max_chunks);
+  if (tid == kIoThread && slot_ok) {  // P and Q' images -> workspace slot
     bulk_s2g(slot + SLOT_P, sX + X_PI, 32768);
     bulk_s2g(slot + SLOT_QP, sX + X_QPI, 16384);
+  }
+  if (tid == kIoThread) {
     bulk_commit();
     if (CHANNEL && next < total) load_qk(next, ce_next, true);  // Q' has read the q tile
   }
@@ -1411,7 +1416,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (tid == kIoThread) {  // Qc and O_intra images -> workspace slot
+  if (tid == kIoThread && slot_ok) {  // Qc and O_intra images -> workspace slot
     bulk_s2g(slot + SLOT_QC, sX + X_QCI, 32768);
     bulk_s2g(slot + SLOT_OI, sX + X_OII, 16384);
     bulk_commit();
@@ -1545,8 +1550,9 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
     sT = nullptr;
   }
   const size_t state_base = ((size_t)sslot * H_v + h) * DK * DK + (size_t)sl * NS;
-  auto slot_of = [&](int u) {
-    return slots + ((size_t)(c_begin + u) * H_v + h) * SLOT_BYTES;
+  auto slot_of = [&](int u) {  // (slot 0 in place of one outside the table: counted, not read)
+    const bool ok = GDR_IN_BOUNDS((int64_t)c_begin + u < chunks.max_chunks);
+    return slots + (ok ? ((size_t)(c_begin + u) * H_v + h) * SLOT_BYTES : 0);
   };
 
   if (warp == kScanLoadWarp) {
@@ -1728,7 +1734,7 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
         }
       }
       mbar_arrive(&empty[st]);
-      if (t < ce.len) {
+      if (t < ce.len && GDR_IN_BOUNDS((int64_t)ce.start + t < chunks.T_total)) {
         uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(ce.start + t) * H_v + h) * DK + sl * NS);
 #pragma unroll
         for (int q = 0; q < NS / 8; ++q) dst[q] = out[q];
@@ -1775,6 +1781,8 @@ bool make_map(CUtensorMap *m, const void *base, CUtensorMapDataType dt, int esiz
 
 }  // namespace
 
+GDR_DEFINE_OOB_COUNTER(oob_count_prefill_tc)
+
 size_t prefill_workspace_bytes(int T, int H_v, int d_k, int d_v, int num_seqs, bool bf16) {
   if (!(bf16 && d_k == DK && d_v == DK))
     return kHeaderBytes + align_up(sizeof(int32_t) * ((size_t)num_seqs + 1), 256);
@@ -1811,7 +1819,7 @@ cudaError_t launch_prefill_tc(const PrefillArgs &a, cudaStream_t stream) {
   }
 
   // a dense batch needs no planning: its chunks follow from the shape
-  Chunks chunks{tab, seq_off, order, 0, 0};
+  Chunks chunks{tab, seq_off, order, 0, 0, T_total, max_chunks};
   cudaError_t e = cudaSuccess;
   if (a.cu_seqlens) {
     TraceScope tr("plan_kernel", stream);

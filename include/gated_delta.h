@@ -318,6 +318,24 @@ KDA_API kda_status_t kda_check_device_status(const void *workspace, void *stream
  * for a NULL workspace) before touching the device.  Asynchronous on `stream`. */
 KDA_API kda_status_t kda_selftest_wait_timeout(void *workspace, int32_t max_polls, void *stream);
 
+/* Bounds-checked build (libgated_delta_checked.so, compiled with
+ * -DGDR_BOUNDS_CHECK; the sanitizer substitute of this library).  In that
+ * build every index a kernel computes for a global-memory access of its own
+ * (inputs, outputs, states, chunk table, workspace slots; the tensor-map tile
+ * copies are bounded by the TMA unit itself) is compared with the extent of
+ * the buffer it addresses.  A failed comparison counts one violation and the
+ * access is skipped: no trap, no access outside the buffer.  Results are
+ * otherwise the same as the normal build's, a little slower.
+ *
+ * kda_bounds_checked(): 1 in the bounds-checked build, 0 in the normal one.
+ *
+ * kda_bounds_violations(): waits for `stream`, then stores in *count the
+ * violations counted on the current device since the last call (and resets
+ * the counters).  Always 0 in the normal build.  Returns KDA_ERR_INVALID_ARG
+ * for a NULL count, KDA_ERR_CUDA if the device cannot be read. */
+KDA_API int32_t kda_bounds_checked(void);
+KDA_API kda_status_t kda_bounds_violations(void *stream, uint32_t *count);
+
 /* Static text for a status code. */
 KDA_API const char *kda_status_string(kda_status_t status);
 

@@ -180,3 +180,16 @@ def test_selftest_wait_timeout_validates_on_host():
     dummy = ctypes.c_void_p(256)  # never dereferenced: the bound check fails first
     assert L.kda_selftest_wait_timeout(dummy, 0, None) == gdr.KDA_ERR_INVALID_ARG
     assert L.kda_selftest_wait_timeout(dummy, 5000, None) == gdr.KDA_ERR_INVALID_ARG
+
+
+def test_checked_build_exports_the_same_symbols():
+    """The bounds-checked build is the same library: same symbols, same ABI."""
+    L = ctypes.CDLL(gdr.checked_library_path)
+    for name in _declared_symbols():
+        assert hasattr(L, name), name
+    with gdr.use_library(gdr.checked_library_path) as C:
+        assert C.kda_abi_version() == 1
+        assert gdr.bounds_checked()
+        assert C.kda_bounds_violations(None, None) == gdr.KDA_ERR_INVALID_ARG
+    assert not gdr.bounds_checked()
+    assert gdr.lib().kda_bounds_violations(None, None) == gdr.KDA_ERR_INVALID_ARG
