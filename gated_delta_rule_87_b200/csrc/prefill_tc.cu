@@ -46,9 +46,9 @@
 //            state), walking the chunks in order: the fp32 state rows in
 //            registers of 4 chain warps, its bf16 copy in shared memory as
 //            the MN-major B operand; per chunk one MMA P S (M = 128, N = the
-//            slice width, K = 128) and one Q' S (M padded to 128), then
+//            slice width, K = 128) and one Q' S (M = 64), then
 //            S <- P S + Qc and o = Q' S + O_intra, with a load warp
-//            streaming the slots through 2-3 stages and 2 output warps.
+//            streaming the slots through 2-3 stages and 4 output warps.
 #include <cudaTypedefs.h>
 
 #include <mutex>
@@ -1457,15 +1457,16 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 // the left), so a (sequence, v-head) chain is split into 128 / NS column
 // slices, one CTA each.  Per chunk u a CTA computes, for its NS columns,
 //     S_{u+1} = P_u S_u + Qc_u        o_u = Q'_u S_u + O_intra_u
-// with S_u in bf16 as the MN-major B operand in shared memory, P_u (K-major)
-// and Q'_u (MN-major, M padded to 128: rows t >= 64 read the next bytes of the
-// stage and land in TMEM lanes nobody reads) as A operands, fp32 accumulators
-// in TMEM and the fp32 state in registers of the chain warps.  Roles,
-// connected by mbarriers:
+// with S_u in bf16 as the MN-major B operand in shared memory, P_u (K-major,
+// M = 128) and Q'_u (MN-major, M = 64) as A operands, fp32 accumulators in
+// TMEM and the fp32 state in registers of the chain warps.  Roles, connected
+// by mbarriers:
 //   chain warps 0-3 : S_{u+1} = (P S)_u + Qc_u, row i = TMEM lane i
-//   output warps 4-5: o_u = (Q' S)_u + O_intra_u, row t = TMEM lane t
-//   MMA warp 6      : the two products of each chunk
-//   load warp 7     : chunk slots into kStages stages (bulk copies)
+//   output warps 4-7: o_u = (Q' S)_u + O_intra_u; an M = 64 product leaves
+//                     rows 16 q .. 16 q + 15 in TMEM lanes 32 q .. 32 q + 15,
+//                     so warp 4 + q (lane quarter q) stores them from lanes 0-15
+//   MMA warp 8      : the two products of each chunk
+//   load warp 9     : chunk slots into kStages stages (bulk copies)
 template <int NS>
 struct ScanCfg {
   static constexpr int kSlices = NS / 32;   // 32-column image slices per CTA
@@ -1481,9 +1482,9 @@ struct ScanCfg {
   static constexpr uint32_t TD_S = 0, TD_O = NS;          // TMEM columns: (P S), (Q' S) x 2
   static constexpr uint32_t TMEM_COLS = NS == 32 ? 128 : 256;
 };
-constexpr int kScanThreads = 256;
-constexpr int kScanMmaWarp = 6, kScanLoadWarp = 7;
-constexpr uint32_t kScanEmptyCount = 128 + 64 + 1;  // chain + output threads + MMA commit
+constexpr int kScanThreads = 320;
+constexpr int kScanMmaWarp = 8, kScanLoadWarp = 9;
+constexpr uint32_t kScanEmptyCount = 128 + 128 + 1;  // chain + output threads + MMA commit
 
 // byte offset of the 16-byte chunk `ch` of state-operand row c (MN-major, NS columns)
 template <int NS>
@@ -1533,7 +1534,7 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
     for (int b = 0; b < 2; ++b) {
       mbar_init(&sb_ready[b], 128);
       mbar_init(&do_full[b], 1);
-      mbar_init(&do_free[b], 64);
+      mbar_init(&do_free[b], 128);
     }
     mbar_init(ds_full, 1);
     mbar_init(drain, 1);
@@ -1590,7 +1591,7 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
     // The whole warp runs the loop and computes the operand descriptors
     // (warp-uniform values); one elected lane issues the products.
     constexpr uint32_t idS = idesc_bf16(128, NS, false, true);  // P K-major, S MN-major
-    constexpr uint32_t idO = idesc_bf16(128, NS, true, true);   // Q' MN-major, S MN-major
+    constexpr uint32_t idO = idesc_bf16(64, NS, true, true);    // Q' MN-major, S MN-major, M = 64
     for (int u = 0; u < nch; ++u) {
       const int st = u % S, b = u & 1;
       if (!mbar_wait_warp(&full[st], (u / S) & 1, err, KDA_DEVICE_TIMEOUT)) break;
@@ -1695,9 +1696,12 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
         *reinterpret_cast<float4 *>(sT + state_base + (size_t)i * DK + j) =
             make_float4(Sr[j], Sr[j + 1], Sr[j + 2], Sr[j + 3]);
     }
-  } else if (warp < 6) {
+  } else if (warp < 8) {
     // ---------------- outputs: row t of o = Q' S + O_intra ----------------
-    const int t = 32 * (warp - 4) + lane;  // TMEM lane quarter warp % 4 = warp - 4
+    // M = 64 product: rows 16 q4 .. +15 in TMEM lanes 32 q4 .. +15 (lane quarter q4 = warp % 4)
+    const int q4 = warp - 4;
+    const bool row_lane = lane < 16;
+    const int t = 16 * q4 + (row_lane ? lane : 0);
     ChunkEntry ce = nch > 0 ? chunks.entry(c_begin) : ChunkEntry{0, 0, 0, 0};
     for (int u = 0; u < nch; ++u) {
       const int st = u % S, b = u & 1;
@@ -1708,7 +1712,7 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
 #pragma unroll
       for (int p = 0; p < NS / 32; ++p) {
         float w32[32];
-        tmem_ld32(taddr(tm, 32 * (warp - 4), Cfg::TD_O + NS * b + 32 * p), w32);
+        tmem_ld32(taddr(tm, 32 * q4, Cfg::TD_O + NS * b + 32 * p), w32);
         tmem_ld_wait();
 #pragma unroll
         for (int e = 0; e < 32; ++e) v[32 * p + e] = w32[e];
@@ -1734,7 +1738,7 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
         }
       }
       mbar_arrive(&empty[st]);
-      if (t < ce.len && GDR_IN_BOUNDS((int64_t)ce.start + t < chunks.T_total)) {
+      if (row_lane && t < ce.len && GDR_IN_BOUNDS((int64_t)ce.start + t < chunks.T_total)) {
         uint4 *dst = reinterpret_cast<uint4 *>(o + ((size_t)(ce.start + t) * H_v + h) * DK + sl * NS);
 #pragma unroll
         for (int q = 0; q < NS / 8; ++q) dst[q] = out[q];
