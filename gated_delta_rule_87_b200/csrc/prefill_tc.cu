@@ -25,8 +25,11 @@
 // sub-chunking", row "KDA") are split at the end E_J of the key's 16-token
 // sub-chunk J:  e^{x_i - G_j} = e^{x_i - E_J} * e^{E_J - G_j}.  The key-side
 // factor is <= 1; the query/key-row factor is <= 1 for rows in later
-// sub-chunks and at most e^{16 |g|max} inside the diagonal sub-chunk, which
-// stays in fp32/bf16 range for per-token log-decays g >= -5.
+// sub-chunks and at most 1/(the key sub-chunk's decay product) inside the
+// diagonal one.  A chunk whose 16-token log-decay sum falls below -64 in some
+// channel takes its Grams from directly formed pair factors instead (fp32,
+// every factor <= 1, out of line), so no gate strength leaves the fp32/bf16
+// range.
 //
 // With the decay applied before the erase (the variant order (I - beta k
 // k^T) Diag(a) S), recall reads the state along a_t . k_t: the erase
