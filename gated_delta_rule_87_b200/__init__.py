@@ -25,6 +25,7 @@ __all__ = [
     "gdn_decode_step", "kda_recurrent_fwd", "gdn_recurrent_fwd", "state_gather", "state_scatter",
     "chunk_workspace_size", "check_device_status", "EXPORTED_SYMBOLS",
     "checked_library_path", "use_library", "bounds_checked", "bounds_violations",
+    "kda_chunk_fwd_host",
     "trace_enable", "trace_read", "ERASE_THEN_DECAY", "DECAY_THEN_ERASE",
     "KDA_OK", "KDA_ERR_INVALID_ARG", "KDA_ERR_UNSUPPORTED", "KDA_ERR_CUDA",
     "KDA_ERR_DEVICE_CHECK", "KDA_ERR_WORKSPACE",
@@ -51,7 +52,7 @@ EXPORTED_SYMBOLS = (
     "kda_trace_enable", "kda_trace_read", "kda_chunk_fwd_noalloc", "kda_chunk_fwd_ex",
     "gdn_chunk_fwd_ex", "kda_recurrent_fwd", "gdn_recurrent_fwd", "kda_state_gather",
     "kda_state_scatter", "kda_selftest_wait_timeout", "kda_bounds_checked",
-    "kda_bounds_violations",
+    "kda_bounds_violations", "kda_chunk_fwd_host", "kda_chunk_fwd_host_buffer_size",
 )
 
 _lock = threading.Lock()
@@ -81,6 +82,8 @@ _SIGS = {
     "kda_chunk_fwd_noalloc": ([_vp] * 9 + [_i32] * 6 + [ctypes.c_int, _vp], ctypes.c_int),
     "kda_trace_read": ([ctypes.c_char_p, _i32, ctypes.POINTER(ctypes.c_float), _i32], _i32),
     "kda_bounds_checked": ([], _i32),
+    "kda_chunk_fwd_host_buffer_size": ([_i32] * 5 + [ctypes.c_int, _i32], _sz),
+    "kda_chunk_fwd_host": ([_vp] * 8 + [_i32] * 5 + [ctypes.c_int, _i32, _vp, _sz, _vp], ctypes.c_int),
     "kda_bounds_violations": ([_vp, ctypes.POINTER(ctypes.c_uint32)], ctypes.c_int),
 }
 
@@ -179,6 +182,16 @@ def _ptr(t) -> Optional[int]:
         return None
     if not t.is_cuda:
         raise ValueError("tensors must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError("tensors must be contiguous")
+    return t.data_ptr()
+
+
+def _host_ptr(t) -> Optional[int]:
+    if t is None:
+        return None
+    if t.is_cuda:
+        raise ValueError("tensors must live in host memory")
     if not t.is_contiguous():
         raise ValueError("tensors must be contiguous")
     return t.data_ptr()
@@ -294,6 +307,36 @@ def kda_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *,
     return _chunk_fwd("channel", q, k, v, g, beta, initial_state, cu_seqlens,
                       output_final_state, o, final_state, workspace, stream, order, state_pool,
                       state_slots)
+
+
+def kda_chunk_fwd_host(q, k, v, g, beta, initial_state=None, *, o, final_state=None,
+                       device_buffer=None, pieces: int = 4, stream=None, device=None):
+    """KDA prefill from pinned HOST tensors (dense batch; layouts as
+    kda_chunk_fwd), the copies overlapped with the kernels (see the C call).
+    ``o`` (and ``final_state`` if given) are host tensors the results land in
+    once the stream is synchronised.  ``device_buffer`` (uint8, on the device)
+    is allocated when None.  Returns the device buffer (its first bytes hold
+    the status word for check_device_status)."""
+    torch = _torch()
+    if q.is_cuda or o.is_cuda:
+        raise ValueError("kda_chunk_fwd_host takes host tensors")
+    B, T, H, d_k = q.shape
+    d_v = v.shape[3]
+    io = _dtype_code(q)
+    _f32(g, "g"), _f32(beta, "beta"), _f32(initial_state, "initial_state")
+    _f32(final_state, "final_state")
+    dev = torch.device("cuda", torch.cuda.current_device()) if device is None else device
+    L = lib()
+    need = int(L.kda_chunk_fwd_host_buffer_size(B, T, H, d_k, d_v, io, pieces))
+    if device_buffer is None or device_buffer.numel() < need:
+        device_buffer = torch.empty(need, dtype=torch.uint8, device=dev)
+    sh = _stream_handle(stream, dev)
+    hp = _host_ptr
+    _check(L.kda_chunk_fwd_host(hp(q), hp(k), hp(v), hp(g), hp(beta), hp(o),
+                                hp(initial_state), hp(final_state), B, T, H, d_k, d_v, io,
+                                pieces, _ptr(device_buffer), device_buffer.numel(), sh),
+           "kda_chunk_fwd_host")
+    return device_buffer
 
 
 def gdn_chunk_fwd(q, k, v, g, beta, initial_state=None, cu_seqlens=None, *,

@@ -4,7 +4,9 @@
 #include <stdio.h>
 #include <string.h>
 
+#include <mutex>
 #include <string>
+#include <vector>
 
 #include "common.cuh"
 #include "gated_delta.h"
@@ -77,11 +79,14 @@ bool use_tensor_core_path(const gdr::PrefillArgs &a) {
   return a.bf16 && a.d_k == 128 && a.d_v == 128;
 }
 
-kda_status_t run_prefill(gdr::PrefillArgs &a, cudaStream_t s) {
+// reset_status false: a later piece of one streamed prefill, which keeps the
+// status word its first piece reset (so that an error of any piece stays
+// recorded, and the kernels of the pieces after it skip their work).
+kda_status_t run_prefill(gdr::PrefillArgs &a, cudaStream_t s, bool reset_status = true) {
   kda_status_t st = check_prefill(a);
   if (st != KDA_OK) return st;
   int32_t *status = reinterpret_cast<int32_t *>(a.workspace);
-  cudaError_t e = cudaMemsetAsync(status, 0, kStatusBytes, s);
+  cudaError_t e = reset_status ? cudaMemsetAsync(status, 0, kStatusBytes, s) : cudaSuccess;
   if (e != cudaSuccess) return cuda_fail(e, "cudaMemsetAsync(status)");
   if (!a.cu_seqlens) a.num_seqs = a.B;
   if (!a.state_slots) a.num_slots = a.num_seqs;
@@ -115,6 +120,64 @@ kda_status_t run_prefill(gdr::PrefillArgs &a, cudaStream_t s) {
   if (e != cudaSuccess) return cuda_fail(e, "prefill launch");
   return KDA_OK;
 }
+
+// ---- prefill from host memory, copies overlapped with the kernels ----
+// Streams and events of the streamed prefill, per device, created once.
+struct HostStreams {
+  cudaStream_t h2d = nullptr, d2h = nullptr;
+  std::vector<cudaEvent_t> ev;
+};
+constexpr int kMaxHostDevices = 64;
+constexpr int kMaxPieces = 64;
+std::mutex g_host_mu;
+HostStreams g_host_streams[kMaxHostDevices];
+
+cudaError_t host_streams(int dev, size_t n_events, HostStreams **out) {
+  HostStreams &h = g_host_streams[dev];
+  cudaError_t e = cudaSuccess;
+  if (!h.h2d) e = cudaStreamCreateWithFlags(&h.h2d, cudaStreamNonBlocking);
+  if (e == cudaSuccess && !h.d2h) e = cudaStreamCreateWithFlags(&h.d2h, cudaStreamNonBlocking);
+  while (e == cudaSuccess && h.ev.size() < n_events) {
+    cudaEvent_t ev;
+    e = cudaEventCreateWithFlags(&ev, cudaEventDisableTiming);
+    if (e == cudaSuccess) h.ev.push_back(ev);
+  }
+  *out = &h;
+  return e;
+}
+
+size_t up256(size_t x) { return (x + 255) / 256 * 256; }
+
+// Device buffer of the streamed prefill: the workspace of one piece first (its
+// status word at offset 0), then q, k, v, g, beta and o with the pieces one
+// after the other ([B, piece length, H, d] each), the initial state and two
+// states the pieces hand over through.
+struct HostLayout {
+  int piece, pieces;
+  size_t q, k, v, g, beta, o, s0, st0, st1, total;
+};
+HostLayout host_layout(int B, int T, int H, int d_k, int d_v, bool bf16, int pieces) {
+  HostLayout L{};
+  const int per = (T + pieces - 1) / pieces;
+  L.piece = (per + gdr::kChunk - 1) / gdr::kChunk * gdr::kChunk;
+  L.pieces = (T + L.piece - 1) / L.piece;
+  const size_t e = bf16 ? 2 : 4, rows = (size_t)B * T * H;
+  const size_t state = (size_t)B * H * d_k * d_v * 4;
+  size_t off = up256(gdr::prefill_workspace_bytes(B * L.piece, H, d_k, d_v, B, bf16));
+  L.q = off; off = up256(off + rows * d_k * e);
+  L.k = off; off = up256(off + rows * d_k * e);
+  L.v = off; off = up256(off + rows * d_v * e);
+  L.g = off; off = up256(off + rows * d_k * 4);
+  L.beta = off; off = up256(off + rows * 4);
+  L.o = off; off = up256(off + rows * d_v * e);
+  L.s0 = off; off = up256(off + state);
+  L.st0 = off; off = up256(off + state);
+  L.st1 = off; off = up256(off + state);
+  L.total = off;
+  return L;
+}
+
+int host_pieces(int32_t pieces) { return pieces <= 0 ? 4 : pieces; }
 
 }  // namespace
 
@@ -214,6 +277,117 @@ kda_status_t kda_chunk_fwd(const void *q, const void *k, const void *v, const fl
   return kda_chunk_fwd_ex(q, k, v, g, beta, o, initial_state, final_state, nullptr, 0,
                           cu_seqlens, num_seqs, B, T, H, d_k, d_v, KDA_ERASE_THEN_DECAY, io_dtype,
                           workspace, workspace_bytes, stream);
+}
+
+size_t kda_chunk_fwd_host_buffer_size(int32_t B, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                      kda_dtype_t io_dtype, int32_t pieces) {
+  if (B <= 0 || T <= 0 || H <= 0 || pieces > kMaxPieces) return 0;
+  return host_layout(B, T, H, d_k, d_v, io_dtype == KDA_BF16, host_pieces(pieces)).total;
+}
+
+kda_status_t kda_chunk_fwd_host(const void *q, const void *k, const void *v, const float *g,
+                                const float *beta, void *o, const float *initial_state,
+                                float *final_state, int32_t B, int32_t T, int32_t H, int32_t d_k,
+                                int32_t d_v, kda_dtype_t io_dtype, int32_t pieces,
+                                void *device_buffer, size_t device_buffer_bytes, void *stream) {
+  if (io_dtype != KDA_F32 && io_dtype != KDA_BF16)
+    return fail(KDA_ERR_INVALID_ARG, "io_dtype must be KDA_F32 or KDA_BF16");
+  if (B <= 0 || T <= 0 || H <= 0)
+    return fail(KDA_ERR_INVALID_ARG, "need B > 0, T > 0, H > 0 (B=%d T=%d H=%d)", B, T, H);
+  if (!head_dim_ok(d_k) || !head_dim_ok(d_v))
+    return fail(KDA_ERR_UNSUPPORTED, "d_k and d_v must be 64 or 128 (got %d, %d)", d_k, d_v);
+  if (pieces > kMaxPieces) return fail(KDA_ERR_INVALID_ARG, "pieces must be <= %d", kMaxPieces);
+  if (!q || !k || !v || !g || !beta || !o)
+    return fail(KDA_ERR_INVALID_ARG, "q, k, v, g, beta and o must be non-NULL");
+  const bool bf16 = io_dtype == KDA_BF16;
+  const HostLayout L = host_layout(B, T, H, d_k, d_v, bf16, host_pieces(pieces));
+  if (!device_buffer || (reinterpret_cast<uintptr_t>(device_buffer) & 255u) ||
+      device_buffer_bytes < L.total)
+    return fail(KDA_ERR_WORKSPACE,
+                "device_buffer must be 256-byte aligned and hold kda_chunk_fwd_host_buffer_size() "
+                "= %zu bytes (got %zu)", L.total, device_buffer_bytes);
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  if (dev < 0 || dev >= kMaxHostDevices) return fail(KDA_ERR_INVALID_ARG, "device %d", dev);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  unsigned char *buf = static_cast<unsigned char *>(device_buffer);
+  const size_t e_io = bf16 ? 2 : 4, state = (size_t)B * H * d_k * d_v * 4;
+  const size_t rq = (size_t)H * d_k * e_io, rv = (size_t)H * d_v * e_io, rg = (size_t)H * d_k * 4,
+               rb = (size_t)H * 4;  // bytes per token row
+
+  std::lock_guard<std::mutex> lk(g_host_mu);
+  HostStreams *hs = nullptr;
+  e = host_streams(dev, 2 * (size_t)L.pieces + 2, &hs);
+  if (e != cudaSuccess) return cuda_fail(e, "creating the copy streams");
+  cudaEvent_t start = hs->ev[0], end = hs->ev[1];
+  // copies start after the work already queued on the caller's stream
+  e = cudaEventRecord(start, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(hs->h2d, start, 0);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(hs->d2h, start, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "ordering the copy streams");
+  // one piece's token rows [t0, t0 + len) of every sequence, host [B, T, row] <-> device [B, len, row]
+  // (one sequence: a plain copy; several: one strided copy)
+  auto h2d = [&](size_t dst_off, const void *src, size_t row, int t0, int len) {
+    unsigned char *dst = buf + dst_off + (size_t)B * t0 * row;
+    const unsigned char *from = static_cast<const unsigned char *>(src) + (size_t)t0 * row;
+    if (B == 1) return cudaMemcpyAsync(dst, from, (size_t)len * row, cudaMemcpyHostToDevice, hs->h2d);
+    return cudaMemcpy2DAsync(dst, (size_t)len * row, from, (size_t)T * row, (size_t)len * row, B,
+                             cudaMemcpyHostToDevice, hs->h2d);
+  };
+  if (initial_state) {
+    e = cudaMemcpyAsync(buf + L.s0, initial_state, state, cudaMemcpyHostToDevice, hs->h2d);
+    if (e != cudaSuccess) return cuda_fail(e, "initial state copy");
+  }
+  for (int p = 0; p < L.pieces; ++p) {
+    const int t0 = p * L.piece, len = T - t0 < L.piece ? T - t0 : L.piece;
+    cudaEvent_t in = hs->ev[2 + 2 * p], done = hs->ev[3 + 2 * p];
+    e = h2d(L.q, q, rq, t0, len);
+    if (e == cudaSuccess) e = h2d(L.k, k, rq, t0, len);
+    if (e == cudaSuccess) e = h2d(L.v, v, rv, t0, len);
+    if (e == cudaSuccess) e = h2d(L.g, g, rg, t0, len);
+    if (e == cudaSuccess) e = h2d(L.beta, beta, rb, t0, len);
+    if (e == cudaSuccess) e = cudaEventRecord(in, hs->h2d);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, in, 0);
+    if (e != cudaSuccess) return cuda_fail(e, "input copy");
+    gdr::PrefillArgs a{};
+    const size_t r0 = (size_t)B * t0;
+    a.q = buf + L.q + r0 * rq; a.k = buf + L.k + r0 * rq; a.v = buf + L.v + r0 * rv;
+    a.g = reinterpret_cast<const float *>(buf + L.g + r0 * rg);
+    a.beta = reinterpret_cast<const float *>(buf + L.beta + r0 * rb);
+    a.o = buf + L.o + r0 * rv;
+    a.initial_state = p > 0 ? reinterpret_cast<const float *>(buf + ((p - 1) & 1 ? L.st1 : L.st0))
+                      : initial_state ? reinterpret_cast<const float *>(buf + L.s0) : nullptr;
+    a.final_state = reinterpret_cast<float *>(buf + (p & 1 ? L.st1 : L.st0));
+    a.num_seqs = B;
+    a.B = B; a.T = len; a.H_qk = H; a.H_v = H; a.d_k = d_k; a.d_v = d_v;
+    a.channel_gate = true; a.bf16 = bf16;
+    a.workspace = buf; a.workspace_bytes = L.q;
+    const kda_status_t st = run_prefill(a, s, p == 0);
+    if (st != KDA_OK) return st;
+    e = cudaEventRecord(done, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(hs->d2h, done, 0);
+    if (e == cudaSuccess && B == 1)
+      e = cudaMemcpyAsync(static_cast<unsigned char *>(o) + (size_t)t0 * rv, buf + L.o + r0 * rv,
+                          (size_t)len * rv, cudaMemcpyDeviceToHost, hs->d2h);
+    else if (e == cudaSuccess)
+      e = cudaMemcpy2DAsync(static_cast<unsigned char *>(o) + (size_t)t0 * rv, (size_t)T * rv,
+                            buf + L.o + r0 * rv, (size_t)len * rv, (size_t)len * rv, B,
+                            cudaMemcpyDeviceToHost, hs->d2h);
+    if (e != cudaSuccess) return cuda_fail(e, "output copy");
+  }
+  if (final_state) {
+    e = cudaMemcpyAsync(final_state, buf + ((L.pieces - 1) & 1 ? L.st1 : L.st0), state,
+                        cudaMemcpyDeviceToHost, hs->d2h);
+    if (e != cudaSuccess) return cuda_fail(e, "final state copy");
+  }
+  // the caller's stream continues once every copy has landed
+  e = cudaEventRecord(end, hs->d2h);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, end, 0);
+  if (e == cudaSuccess) e = cudaEventRecord(end, hs->h2d);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, end, 0);
+  if (e != cudaSuccess) return cuda_fail(e, "joining the copy streams");
+  return KDA_OK;
 }
 
 kda_status_t gdn_chunk_fwd_ex(const void *q, const void *k, const void *v, const float *g,

@@ -299,6 +299,52 @@ KDA_API kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, const v
                                            int32_t B, int32_t T, int32_t H, int32_t d_k,
                                            int32_t d_v, kda_dtype_t io_dtype, void *stream);
 
+/* ---------------------------------------------------------------------------
+ * kda_chunk_fwd_host -- the KDA prefill of kda_chunk_fwd (dense batch, same
+ * operator, same kernels) with q, k, v, g, beta, o and the states in HOST
+ * memory, for a caller whose prompt is not on the device yet.  The tokens are
+ * cut into `pieces` spans of equal length (a multiple of C = 64; pieces <= 0
+ * means 4, at most 64): while the kernels run on span p, the host-to-device
+ * copy of span p + 1 and the device-to-host copy of span p - 1's output run
+ * on two internal copy streams, so the transfers overlap each other and the
+ * computation.  Each span is one prefill whose initial state is the previous
+ * span's final state (fp32, through device memory), which is what a single
+ * call over all tokens computes between its chunks: the results equal
+ * kda_chunk_fwd's.
+ *
+ *   q, k, v, g, beta, o, initial_state, final_state
+ *                 host pointers, the layouts of kda_chunk_fwd; pinned memory
+ *                 (cudaHostAlloc / cudaHostRegister) for the copies to
+ *                 overlap; initial_state may be NULL (zeros), final_state
+ *                 NULL (not returned)
+ *   B, T, H, d_k, d_v, io_dtype    as kda_chunk_fwd; T > 0
+ *   device_buffer  device memory of kda_chunk_fwd_host_buffer_size() bytes,
+ *                 256-byte aligned, owned by the caller: the staged inputs
+ *                 and outputs, the states and the workspace, whose status
+ *                 word is at offset 0 (read it with kda_check_device_status
+ *                 on device_buffer)
+ *   stream        the caller's stream: the kernels run on it, the copies
+ *                 start after the work queued on it before the call, and work
+ *                 queued after the call starts once every copy has landed
+ *
+ * Asynchronous like the other calls: o and final_state are valid on the host
+ * once `stream` has been synchronised.  Calls for one device serialise their
+ * enqueueing on an internal lock (the copy streams are shared per device).
+ * Returns KDA_ERR_INVALID_ARG / KDA_ERR_UNSUPPORTED for bad arguments (T = 0
+ * included: there is nothing to stream), KDA_ERR_WORKSPACE for a missing,
+ * misaligned or short device_buffer, KDA_ERR_CUDA for a failed copy or
+ * launch.
+ * ------------------------------------------------------------------------ */
+KDA_API size_t kda_chunk_fwd_host_buffer_size(int32_t B, int32_t T, int32_t H, int32_t d_k,
+                                              int32_t d_v, kda_dtype_t io_dtype, int32_t pieces);
+KDA_API kda_status_t kda_chunk_fwd_host(const void *q, const void *k, const void *v,
+                                        const float *g, const float *beta, void *o,
+                                        const float *initial_state, float *final_state,
+                                        int32_t B, int32_t T, int32_t H, int32_t d_k, int32_t d_v,
+                                        kda_dtype_t io_dtype, int32_t pieces,
+                                        void *device_buffer, size_t device_buffer_bytes,
+                                        void *stream);
+
 /* Wait for `stream`, then read the device status word of a prefill workspace.
  * Returns KDA_OK or KDA_ERR_DEVICE_CHECK (device code in *device_code when
  * non-NULL), or KDA_ERR_CUDA.  Synchronises the stream. */

@@ -193,3 +193,35 @@ def test_checked_build_exports_the_same_symbols():
         assert C.kda_bounds_violations(None, None) == gdr.KDA_ERR_INVALID_ARG
     assert not gdr.bounds_checked()
     assert gdr.lib().kda_bounds_violations(None, None) == gdr.KDA_ERR_INVALID_ARG
+
+
+@pytest.mark.parametrize("over,status", [
+    (dict(T=0), gdr.KDA_ERR_INVALID_ARG),
+    (dict(pieces=65), gdr.KDA_ERR_INVALID_ARG),
+    (dict(q=None), gdr.KDA_ERR_INVALID_ARG),
+    (dict(io=7), gdr.KDA_ERR_INVALID_ARG),
+    (dict(d_k=96), gdr.KDA_ERR_UNSUPPORTED),
+    (dict(buf=None), gdr.KDA_ERR_WORKSPACE),
+    (dict(buf=FAKE + 16), gdr.KDA_ERR_WORKSPACE),
+    (dict(buf_bytes=1024), gdr.KDA_ERR_WORKSPACE),
+])
+def test_streamed_prefill_rejects_bad_arguments_on_host(over, status):
+    L = gdr.lib()
+    kw = dict(q=FAKE, B=1, T=256, H=2, d_k=128, d_v=128, io=1, pieces=4, buf=FAKE,
+              buf_bytes=1 << 30)
+    kw.update(over)
+    st = L.kda_chunk_fwd_host(kw["q"], FAKE, FAKE, FAKE, FAKE, FAKE, None, None, kw["B"], kw["T"],
+                              kw["H"], kw["d_k"], kw["d_v"], kw["io"], kw["pieces"], kw["buf"],
+                              kw["buf_bytes"], None)
+    assert st == status
+    assert L.kda_last_error()
+
+
+def test_streamed_prefill_buffer_size():
+    L = gdr.lib()
+    a = L.kda_chunk_fwd_host_buffer_size(1, 4096, 32, 128, 128, 1, 8)
+    b = L.kda_chunk_fwd_host_buffer_size(1, 8192, 32, 128, 128, 1, 8)
+    # at least the staged inputs and output: q, k, v, o bf16 and g fp32 per token-head
+    assert a >= 4096 * 32 * (4 * 128 * 2 + 128 * 4) and b > a
+    assert L.kda_chunk_fwd_host_buffer_size(1, 4096, 32, 128, 128, 1, 65) == 0
+    assert L.kda_chunk_fwd_host_buffer_size(1, 0, 32, 128, 128, 1, 8) == 0

@@ -1,7 +1,8 @@
 """The bounds-checked build (libgated_delta_checked.so, the sanitizer
 substitute): every index its kernels compute for a global access of their own
 is compared with the extent of its buffer; a violation is counted and the
-access skipped.  A selection of the GPU parity tests runs through that build:
+access skipped.  A selection of the GPU parity tests (the four timed workloads at full size
+among them) runs through that build:
 each must still match the oracle and leave the violation count at zero.
 Covers every kernel: the planning kernel, the tensor-core prep and scan, the
 fp32 path, the token-by-token kernel, the state copies."""
@@ -34,6 +35,11 @@ CASES = [
     ("test_gpu_state_pool", "test_prefill_updates_pool_in_place", dict(io="bf16", gate="channel")),
     ("test_gpu_state_pool", "test_gather_scatter_are_exact_copies", {}),
     ("test_gpu_state_pool", "test_empty_prefill_leaves_pool_unchanged", {}),
+    # the timed workloads at full size
+    ("test_gpu_prefill", "test_kda_prefill_full_workload", {}),
+    ("test_gpu_prefill", "test_kda_varlen_full_workload_sampled_heads", {}),
+    ("test_gpu_prefill", "test_gdn_long_full_workload_sampled_heads", {}),
+    ("test_gpu_decode", "test_kda_decode_full_size_sampled", {}),
 ]
 
 
