@@ -40,6 +40,8 @@ CASES = [
     ("test_gpu_prefill", "test_kda_varlen_full_workload_sampled_heads", {}),
     ("test_gpu_prefill", "test_gdn_long_full_workload_sampled_heads", {}),
     ("test_gpu_decode", "test_kda_decode_full_size_sampled", {}),
+    ("test_gpu_host_stream", "test_streamed_prefill_equals_device_call",
+     dict(io="bf16", B=2, T=1000, pieces=3)),
 ]
 
 
