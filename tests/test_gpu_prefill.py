@@ -232,12 +232,14 @@ def test_kda_prefill_full_workload():
 def test_kda_varlen_full_workload_sampled_heads():
     x = W.make_prefill(W.WORKLOADS["kda_varlen"], seed=0)
     assert list(np.diff(x.cu_seqlens)) == [14090, 10808, 8875, 5168, 5752, 1653, 2179, 1277]
-    _check(x, heads=[0, 13, 31], regress=1e-2)
+    # eight heads: every quarter of the head range, both ends
+    _check(x, heads=[0, 5, 9, 13, 18, 22, 27, 31], regress=1e-2)
 
 
 def test_gdn_long_full_workload_sampled_heads():
     x = W.make_prefill(W.WORKLOADS["gdn_long"], seed=0)
-    _check(x, heads=[0, 1, 30], regress=1e-2)
+    # eight v-heads: both v-heads of q/k heads 0 and 15, and four q/k heads between
+    _check(x, heads=[0, 1, 9, 14, 17, 22, 30, 31], regress=1e-2)
 
 
 @pytest.mark.parametrize("nseq", [8, 20])
