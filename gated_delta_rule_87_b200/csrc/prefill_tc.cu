@@ -1310,11 +1310,14 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
   tc_fence_after();
 
-  // ---- 9. thread 32: K_b^T beta W (for P), X = W^T (B_e beta)^T (for Q');
-  //         thread 0: O_intra -= tril(B_e) beta U (M = 128 as in step 6),
-  //         Qc -= (beta K e^{G_L-Gp})^T U (lanes i, columns j) ----
+  // ---- 9. one thread, in this order: K_b^T beta W (for P), X = W^T (B_e beta)^T
+  //         (for Q'), then O_intra -= tril(B_e) beta U (M = 128 as in step 6) and
+  //         Qc -= (beta K e^{G_L-Gp})^T U (lanes i, columns j).  Products issue one
+  //         at a time whatever thread issues them, so a single issuer puts P and
+  //         X, whose readback comes first, ahead of the other two (from two
+  //         threads they interleave: prep 1.2-2.7 % slower) ----
   if (tid == 32) {
-    const uint32_t wsm = smem_u32(sX + X_W);
+    const uint32_t wsm = smem_u32(sX + X_W), usm = smem_u32(sX + X_U);
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_P, desc_mnmajor(smem_u32(sm + OFF_KBB), 16 * kk, 8192), desc_kmajor(wsm, 16 * kk, 0),
@@ -1324,10 +1327,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       mma_bf16(tm + TM_X, desc_kmajor(wsm, 16 * kk, 0), desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0),
                idesc_bf16(128, 64, false, false), kk > 0);
     mma_commit(bar_px);
-  } else if (tid == 0) {
-    const uint32_t usm = smem_u32(sX + X_U);
-    // the first O_intra and Qc terms (thread 288) have completed: warps 8-15
-    // passed bar_yo's phase before the barrier ahead of the W/U round
 #pragma unroll
     for (int kk = 0; kk < 4; ++kk)
       mma_bf16(tm + TM_OI, desc_kmajor(smem_u32(sX + X_BE), 16 * kk, 0), desc_kmajor(usm, 16 * kk, 0),
