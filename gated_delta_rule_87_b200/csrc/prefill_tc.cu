@@ -22,12 +22,14 @@
 // P is the product of the chunk's transition matrices in WY form.
 //
 // Per-channel decay factors inside the Gram sums ("numerical range -- needs
-// sub-chunking", row "KDA") are split at the end E_J of the key's 16-token
-// sub-chunk J:  e^{x_i - G_j} = e^{x_i - E_J} * e^{E_J - G_j}.  The key-side
-// factor is <= 1; the query/key-row factor is <= 1 for rows in later
-// sub-chunks and at most 1/(the key sub-chunk's decay product) inside the
-// diagonal one.  A chunk whose 16-token log-decay sum falls below -64 in some
-// channel takes its Grams from directly formed pair factors instead (fp32,
+// sub-chunking", row "KDA") are split at an anchor, the cumulative log-decay
+// E_1 at the end of the chunk's second 16-token sub-chunk:
+// e^{x_i - G_j} = e^{x_i - E_1} * e^{E_1 - G_j}.  A row factor is at most the
+// inverse decay product of the two sub-chunks up to the anchor, a key factor
+// that of the two after it; bf16 and fp32 rounding is relative, so the scaled
+// operands lose nothing as long as they stay in range.  A chunk with a 16-token
+// log-decay sum below -32 in some channel (so that a 32-token one could fall
+// below -64) takes its Grams from directly formed pair factors instead (fp32,
 // every factor <= 1, out of line), so no gate strength leaves the fp32/bf16
 // range.
 //
@@ -244,9 +246,8 @@ constexpr uint32_t PREP_SMEM = OFF_MISC + 14336 + 1024;
 
 // X region, gram phase
 constexpr uint32_t X_R = 0;           // 32 KB, K-major B [128 rows][128], blocks 16 KB apart
-constexpr uint32_t X_LEFT = 32768;    // 48 KB, two overlapped K-major A tiles (anchors E_0, E_2)
-constexpr uint32_t LEFT_BLOCK = 24576;  // 64-column blocks of the left tiles
-constexpr uint32_t LEFT_G1 = 8192;      // anchor-E_2 tile: its rows 64..127 land past the E_0 tile's
+constexpr uint32_t X_LEFT = 32768;    // 48 KB, K-major A tile [128 rows][128] ([K; Q] scaled to the anchor)
+constexpr uint32_t LEFT_BLOCK = 24576;  // its 64-column blocks (16 KB used of each)
 // X region, after the Gram MMAs
 constexpr uint32_t X_AWBW = 0;        // 16 KB K-major B [128 i'][64 j]
 constexpr uint32_t X_BE = 16384;      // 8 KB  K-major B [64 i][64 j]
@@ -254,8 +255,10 @@ constexpr uint32_t X_TINVB = 24576;   // 8 KB  K-major B [64 i][64 j]; scratch b
 constexpr int LDN = 68;               // padded row stride (floats) of the fp32 64x64 tiles
 constexpr uint32_t X_GEXACT = 50176;  // exact Gram only: f32 [65][kLdG] cumulative log-decay
 constexpr int kLdG = 129;             // its padded row stride (floats)
-// A sub-chunk log-decay sum below this sends its item to the exact Gram
-// (e^{64} leaves e^{24} of headroom below the fp32/bf16 maximum for q, k).
+// The Gram's operands grow by at most e^{-(a 32-token log-decay sum)}; this is
+// the bound on that sum (e^{64} leaves e^{24} of headroom below the fp32/bf16
+// maximum for q, k).  An item with a 16-token sum below half of it (so that a
+// 32-token one may fall below it) takes the exact Gram.
 constexpr float kExactBound = -64.f;
 constexpr uint32_t X_NAE = 32768;     // 17 KB f32 [64][LDN]  (N = tril(A_e) diag(beta))
 constexpr uint32_t X_TINVF = 50176;   // 17 KB f32 [64][LDN]  (T^{-1}); both dead after step 6
@@ -712,11 +715,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       sGsum[bI * DK + c2] = s0 + os0;
       sGsum[bI * DK + c2 + 1] = s1 + os1;
     }
-    // The two-anchor Gram scales operands by up to 1/PB (PB: a channel's decay
-    // product over one 16-token sub-chunk).  A sub-chunk whose log-decay sum
-    // is below kExactBound would push them past the fp32/bf16 range: such an
-    // item takes the exact Gram below instead.
-    const bool steep = rh == 0 && (s0 + os0 < kExactBound || s1 + os1 < kExactBound);
+    // The Gram scales operands by up to the inverse decay product of two
+    // 16-token sub-chunks; a sub-chunk whose log-decay sum is below half of
+    // kExactBound could push them past the fp32/bf16 range: such an item takes
+    // the exact Gram below instead.
+    const bool steep = rh == 0 && (s0 + os0 < 0.5f * kExactBound || s1 + os1 < 0.5f * kExactBound);
     if (__any_sync(0xffffffffu, steep) && lane == 0) *s_exact = 1u;  // every writer writes 1
   }
   // the previous item's image copies must have read the X region before it is rebuilt
@@ -740,10 +743,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 
   // ---- 3. one pass builds every operand of the chunk ----
   {
-    // Gram anchors E_0 (key sub-chunks 0, 1) and E_2 (2, 3).  Row factors
-    // F_A = e^{E_{I-1} - E_A} for a row of sub-chunk I >= A: 1/PB_A >= 1 for
-    // I = A, 1 for I = A + 1, products of PB <= 1 beyond; a key of sub-chunk
-    // J = A + 1 takes e^{E_A - E_J} = 1/PB_J on top of its suffix product.
+    // The Gram's anchor is E_1.  A row of sub-chunk I takes e^{E_{I-1} - E_1}
+    // on top of its prefix product (1/(PB_0 PB_1), 1/PB_1, 1, PB_2 for
+    // I = 0 .. 3), a key of sub-chunk I takes e^{E_1 - E_I} on top of its
+    // suffix product (PB_1, 1, 1/PB_2, 1/(PB_2 PB_3)); PB_J is a channel's
+    // decay product over sub-chunk J.
     float ei0 = 1.f, ei1 = 1.f, ge0 = 1.f, ge1 = 1.f;  // e^{E_{I-1}}, e^{G_L - E_I}
 #pragma unroll
     for (int J = 0; J < 4; ++J) {
@@ -756,21 +760,26 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         ge1 *= sPblk[J * DK + c2 + 1];
       }
     }
-    const float inv0 = __expf(-sGsum[bI * DK + c2]), inv1 = __expf(-sGsum[bI * DK + c2 + 1]);  // 1/PB_I
-    float fa0 = 1.f, fa1 = 1.f;  // anchor E_0
+    float fa0, fa1, rf0, rf1;
     if (bI == 0) {
-      fa0 = inv0;
-      fa1 = inv1;
-    } else if (bI >= 2) {
-      fa0 = sPblk[1 * DK + c2];
-      fa1 = sPblk[1 * DK + c2 + 1];
-      if (bI == 3) {
-        fa0 *= sPblk[2 * DK + c2];
-        fa1 *= sPblk[2 * DK + c2 + 1];
-      }
+      fa0 = __expf(-(sGsum[c2] + sGsum[DK + c2]));
+      fa1 = __expf(-(sGsum[c2 + 1] + sGsum[DK + c2 + 1]));
+      rf0 = sPblk[DK + c2];
+      rf1 = sPblk[DK + c2 + 1];
+    } else if (bI == 1) {
+      fa0 = __expf(-sGsum[DK + c2]);
+      fa1 = __expf(-sGsum[DK + c2 + 1]);
+      rf0 = rf1 = 1.f;
+    } else if (bI == 2) {
+      fa0 = fa1 = 1.f;
+      rf0 = __expf(-sGsum[2 * DK + c2]);
+      rf1 = __expf(-sGsum[2 * DK + c2 + 1]);
+    } else {
+      fa0 = sPblk[2 * DK + c2];
+      fa1 = sPblk[2 * DK + c2 + 1];
+      rf0 = __expf(-(sGsum[2 * DK + c2] + sGsum[3 * DK + c2]));
+      rf1 = __expf(-(sGsum[2 * DK + c2 + 1] + sGsum[3 * DK + c2 + 1]));
     }
-    const float fb0 = bI == 2 ? inv0 : 1.f, fb1 = bI == 2 ? inv1 : 1.f;  // anchor E_2
-    const float rf0 = (bI & 1) ? inv0 : 1.f, rf1 = (bI & 1) ? inv1 : 1.f;  // key side
     if (bI == 0 && rh == 0) {
       sGLe[c2] = ge0 * sPblk[c2];  // e^{G_L}: product over all four sub-chunks
       sGLe[c2 + 1] = ge1 * sPblk[c2 + 1];
@@ -787,7 +796,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // Channel pairs in packed fp32x2 arithmetic.  Every operand row written
     // here has the same residue mod 8 as t, so the SW128 position of channel
     // pair c2 within a 128-byte row is one offset per row.
-    const float2 fa = make_float2(fa0, fa1), fb = make_float2(fb0, fb1), rf = make_float2(rf0, rf1);
+    const float2 fa = make_float2(fa0, fa1), rf = make_float2(rf0, rf1);
     const float2 ei = make_float2(ei0, ei1), ge = make_float2(ge0, ge1);
     const uint32_t cblk = (uint32_t)(c2 >> 6), cpos = (uint32_t)(c2 & 63) * 2;  // byte in the row
     unsigned char *const rbase = sX + X_R + cblk * 16384;
@@ -819,16 +828,12 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       const float2 kb = __fmul2_rn(k, bk), qb = __fmul2_rn(q, bq);
       const uint32_t rowK = (uint32_t)(32 * bI + 8 * rh + r) * 128 + x, rowQ = rowK + 16 * 128;
       if (!exact) {  // the exact Gram's images occupy this region
-        // Gram right operand (keys scaled to their group's anchor)
+        // Gram right operand (keys scaled to the anchor)
         st4(rbase + rowK, __fmul2_rn(kw, rf));
         st4(rbase + rowQ, __fmul2_rn(ke, rf));
-        // Gram left operands: anchor E_0 (all rows), anchor E_2 (sub-chunks 2, 3)
+        // Gram left operand (rows scaled to the anchor)
         st4(lbase + rowK, __fmul2_rn(kb, fa));
         st4(lbase + rowQ, __fmul2_rn(qb, fa));
-        if (bI >= 2) {
-          st4(lbase + LEFT_G1 + rowK, __fmul2_rn(kb, fb));
-          st4(lbase + LEFT_G1 + rowQ, __fmul2_rn(qb, fb));
-        }
       }
       // K e^{Gp} over k, q e^{G} over q (same element, same owner), beta K e^{G_L - G|Gp}
       st4(kbase + koff, __fmul2_rn(kb, ei));
@@ -843,21 +848,22 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   __syncthreads();
   tc_fence_after();
 
-  // ---- 4. Gram MMAs: per anchor group A, [K;Q] rows x 64 key columns (w, e of
-  //         two key sub-chunks); one issuing thread per group ----
+  // ---- 4. Gram MMA: [K;Q] rows x 128 key columns (w and e of the four key
+  //         sub-chunks), one M = 128, N = 128 product (the two anchors of an
+  //         earlier form needed two N = 64 products: 8 more issues, prep 4.5 %
+  //         slower) ----
   if (tid == 0) *s_exact = 0u;  // every thread holds its copy of the flag
   if ((tid == 0 || tid == 32) && exact) {
     mbar_arrive(bar_mma);  // the phase completes with no product: the exact Gram is written
-  } else if (tid == 0 || tid == 32) {
-    const int A = tid >> 5;
-    constexpr uint32_t ID = idesc_bf16(128, 64, false, false);
-    const uint32_t a_base = smem_u32(sX + X_LEFT + A * LEFT_G1);
-    const uint32_t r_base = smem_u32(sX + X_R + A * 8192);
+  } else if (tid == 0) {
+    constexpr uint32_t ID = idesc_bf16(128, 128, false, false);
+    const uint32_t a_base = smem_u32(sX + X_LEFT), r_base = smem_u32(sX + X_R);
 #pragma unroll
     for (int kk = 0; kk < 8; ++kk)
-      mma_bf16(tm + TM_GRAM + 64 * A, desc_kmajor(a_base, 16 * kk, LEFT_BLOCK),
+      mma_bf16(tm + TM_GRAM, desc_kmajor(a_base, 16 * kk, LEFT_BLOCK),
                desc_kmajor(r_base, 16 * kk, 16384), ID, kk > 0);
     mma_commit(bar_mma);
+    mma_commit(bar_mma);  // the phase counts two commits
   }
   __syncwarp();
   wait_bar(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);

@@ -97,7 +97,7 @@ typedef enum { KDA_ERASE_THEN_DECAY = 0, KDA_DECAY_THEN_ERASE = 1 } kda_order_t;
  *   g             [B, T, H, d_k]   fp32 log-decay (<= 0; a = exp(g)), any
  *                                  magnitude.  (The bf16 path computes a
  *                                  chunk whose 16-token decay sum falls
- *                                  below -64 in some channel with directly
+ *                                  below -32 in some channel with directly
  *                                  formed pair factors: exact, but slower.)
  *   beta          [B, T, H]        fp32 write strength
  *   o             [B, T, H, d_v]   io_dtype, written

@@ -107,25 +107,29 @@ def test_strong_decay(gate, scale):
     _check(W.make_prefill(w, seed=13))
 
 
-@pytest.mark.parametrize("scale,order", [(4.0, "erase_then_decay"), (8.0, "erase_then_decay"),
-                                         (4.0, "decay_then_erase")])
-def test_kda_steep_decays(scale, order):
-    """Per-token log-decays down to -16 and beyond on the bf16 tensor-core
-    path.  A 16-token sub-chunk whose log-decay sum (for some channel) falls
-    below -64 would push the two-anchor Gram's scale factors past the
-    fp32/bf16 range; the kernel computes such items' Grams exactly instead.
-    At scale 4 both kinds of item occur (the ragged last chunk is not steep),
-    at scale 8 (mean -6.5 per token) every full chunk takes the exact Gram."""
+@pytest.mark.parametrize("scale,order,mixed", [(1.5, "erase_then_decay", True),
+                                               (2.0, "decay_then_erase", True),
+                                               (4.0, "erase_then_decay", False),
+                                               (8.0, "erase_then_decay", False)])
+def test_kda_steep_decays(scale, order, mixed):
+    """Steep per-channel decays on the bf16 tensor-core path.  The Gram scales
+    its operands by up to the inverse decay product of 32 tokens; a chunk with
+    a 16-token log-decay sum below -32 in some channel (so that a 32-token one
+    could fall below -64 and push the operands past the fp32/bf16 range) has
+    its Grams computed exactly instead.  At scales 1.5 and 2 both kinds of
+    chunk occur in one call; at 4 and 8 (per-token log-decays down to -16 and
+    -33) every chunk takes the exact Gram."""
     w = W.WORKLOADS["kda_prefill"].replace(T=200, H_qk=2, H_v=2, gate_scale=scale,
                                            init_state=True)
     x = W.make_prefill(w, seed=17)
-    assert x.g.min() <= -15.0
     # sub-chunk sums of the log-decay per (16-token sub-chunk, head, channel)
     gp = np.zeros((256,) + x.g.shape[1:], np.float64)
     gp[:200] = x.g
     sums = gp.reshape(16, 16, *x.g.shape[1:]).sum(axis=1)
-    steep = (sums < -64.0).any(axis=(-1,)).reshape(4, 4, -1).any(axis=1)  # per (chunk, head)
-    assert steep.any() and (scale > 4 or not steep.all())
+    steep = (sums < -32.0).any(axis=(-1,)).reshape(4, 4, -1).any(axis=1)  # per (chunk, head)
+    assert steep.any() and (not steep.all()) == mixed
+    if not mixed:
+        assert x.g.min() <= -15.0
     _check(x, order=order)
 
 
