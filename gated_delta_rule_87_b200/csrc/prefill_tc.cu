@@ -1600,32 +1600,41 @@ chunk_scan_kernel(const int32_t *hdr, const Chunks chunks, const unsigned char *
     // (warp-uniform values); one elected lane issues the products.
     constexpr uint32_t idS = idesc_bf16(128, NS, false, true);  // P K-major, S MN-major
     constexpr uint32_t idO = idesc_bf16(64, NS, true, true);    // Q' MN-major, S MN-major, M = 64
+    // descriptors of K-slice 0 for every stage and operand buffer, built once;
+    // K-slice kk adds its byte offset / 16 to the start-address field
+    uint64_t dP[S], dQ[S], dS[2];
+#pragma unroll
+    for (int st = 0; st < S; ++st) {
+      const uint32_t stage = smem_u32(sm + st * Cfg::ST_BYTES);
+      dP[st] = desc_kmajor(stage + Cfg::ST_P, 0, 16384);
+      dQ[st] = desc_mnmajor(stage + Cfg::ST_QP, 0, 16384);
+    }
+#pragma unroll
+    for (int b = 0; b < 2; ++b) dS[b] = sop_desc<NS>(smem_u32(sm + Cfg::OFF_SB + b * Cfg::SB_BYTES), 0);
+    constexpr uint32_t kSOp = NS == 32 ? 64 : 128;  // state operand: 16-byte units per K-slice
     for (int u = 0; u < nch; ++u) {
       const int st = u % S, b = u & 1;
       if (!mbar_wait_warp(&full[st], (u / S) & 1, err, KDA_DEVICE_TIMEOUT)) break;
       if (!mbar_wait_warp(&sb_ready[b], (u >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
       tc_fence_after();
-      const uint32_t stage = smem_u32(sm + st * Cfg::ST_BYTES);
-      const uint32_t sb = smem_u32(sm + Cfg::OFF_SB + b * Cfg::SB_BYTES);
-      uint64_t da[8], dbs[8];
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) {
-        da[kk] = desc_kmajor(stage + Cfg::ST_P, 16 * kk, 16384);
-        dbs[kk] = sop_desc<NS>(sb, kk);
-      }
+      const uint64_t p0 = st == 0 ? dP[0] : (st == 1 ? dP[1] : dP[S - 1]);
+      const uint64_t q0 = st == 0 ? dQ[0] : (st == 1 ? dQ[1] : dQ[S - 1]);
+      const uint64_t s0d = b ? dS[1] : dS[0];
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_bf16(tm + Cfg::TD_S, da[kk], dbs[kk], idS, kk > 0);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tm + Cfg::TD_S, p0 + (uint64_t)((kk >> 2) * 1024 + (kk & 3) * 2),
+                   s0d + (uint64_t)(kk * kSOp), idS, kk > 0);
         mma_commit(ds_full);
       }
       __syncwarp();
       if (u >= 2 && !mbar_wait_warp(&do_free[b], ((u - 2) >> 1) & 1, err, KDA_DEVICE_TIMEOUT)) break;
       tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk) da[kk] = desc_mnmajor(stage + Cfg::ST_QP, 16 * kk, 16384);
       if (elect_one()) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) mma_bf16(tm + Cfg::TD_O + NS * b, da[kk], dbs[kk], idO, kk > 0);
+        for (int kk = 0; kk < 8; ++kk)
+          mma_bf16(tm + Cfg::TD_O + NS * b, q0 + (uint64_t)(kk * 128), s0d + (uint64_t)(kk * kSOp),
+                   idO, kk > 0);
         mma_commit(&do_full[b]);
         mma_commit(&empty[st]);
       }
