@@ -329,7 +329,9 @@ KDA_API kda_status_t kda_chunk_fwd_noalloc(const void *q, const void *k, const v
  *
  * Asynchronous like the other calls: o and final_state are valid on the host
  * once `stream` has been synchronised.  Calls for one device serialise their
- * enqueueing on an internal lock (the copy streams are shared per device).
+ * enqueueing on an internal lock (the copy streams are shared per device; the
+ * library creates them and their events at the first call on a device and
+ * keeps them until the process exits).
  * Returns KDA_ERR_INVALID_ARG / KDA_ERR_UNSUPPORTED for bad arguments (T = 0
  * included: there is nothing to stream), KDA_ERR_WORKSPACE for a missing,
  * misaligned or short device_buffer, KDA_ERR_CUDA for a failed copy or
