@@ -240,6 +240,7 @@ constexpr uint32_t MISC_GSUM = 2560;   // f32[4][128] sum of g over each sub-chu
 constexpr uint32_t MISC_GLE = 4608;    // f32[128] e^{G_L}
 constexpr uint32_t MISC_BAR = 5120;    // 5 x u64; the drain barrier at +48, two failure flags at +56
 constexpr uint32_t MISC_TSLOT = 5160;  // u32; the exact-Gram flag at +4
+constexpr uint32_t MISC_GBAR = 5184;   // u64: the gate tile's own TMA barrier (per-channel gate)
 constexpr uint32_t MISC_XP = 6144;     // f32[4][2][128] product of a over each half sub-chunk
 constexpr uint32_t MISC_XS = 10240;    // f32[4][2][128] sum of g over each half sub-chunk
 constexpr uint32_t PREP_SMEM = OFF_MISC + 14336 + 1024;
@@ -503,6 +504,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   uint64_t *bar_px = bar_tma + 3;    // P and X (one commit)
   uint64_t *bar_oq = bar_tma + 4;    // the second O_intra term and Qc (one commit)
   uint64_t *bar_drain = bar_tma + 6;  // after an expired wait: every issuing thread's last MMAs
+  // the gate tile lands on a barrier of its own, so that an item's decays can
+  // start while its q, k, v tiles are still on their way
+  uint64_t *bar_g = reinterpret_cast<uint64_t *>(sm + OFF_MISC + MISC_GBAR);
   uint32_t *tslot = reinterpret_cast<uint32_t *>(sm + OFF_MISC + MISC_TSLOT);
   volatile uint32_t *s_exact = reinterpret_cast<volatile uint32_t *>(sm + OFF_MISC + MISC_TSLOT + 4);
   volatile uint32_t *s_fail = reinterpret_cast<volatile uint32_t *>(sm + OFF_MISC + MISC_BAR + 56);
@@ -522,6 +526,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   if (tid == 0) {
     mbar_init(bar_tma, 1);
+    mbar_init(bar_g, 1);
     mbar_init(bar_mma, 2);
     mbar_init(bar_yo, 2);
     mbar_init(bar_px, 1);
@@ -544,20 +549,25 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // its buffer: g once the decays are taken, v once the products before T^{-1}
   // have run, q and k once their last reader has run (the raw-tile Gram and
   // the image pass with a scalar gate, before v; Q' with a per-channel gate,
-  // after v).  Every load but the last adds its bytes to the phase without an
-  // arrival; the last one arrives, so the phase completes only when every tile
-  // has landed.  All from thread kIoThread, in program order.
+  // after v).  The gate tile completes a phase of its own barrier, waited for at
+  // the top of the item; of the q, k, v loads every one but the last adds its
+  // bytes to the phase without an arrival and the last one arrives, so that
+  // phase completes only when all three have landed.  It is waited for after
+  // the decays, which need the gate alone: the q/k load issued late in the
+  // previous item (after its Q' readback) lands meanwhile.  All from thread
+  // kIoThread, in program order.
   // TMA phases armed by kIoThread (loads whose last one carried the arrival)
   // and whether loads of a phase not yet armed are in flight: an aborted CTA
   // completes and waits out every such phase before it exits.
-  int tma_armed = 0, tma_done = 0;
+  // (bar_g: every gate load is a phase of its own, g_armed of them so far)
+  int tma_armed = 0, tma_done = 0, g_armed = 0, g_done = 0;
   bool tma_partial = false;
   auto load_g = [&](int w, const ChunkEntry &e) {
     if (CHANNEL) {
-      tma_partial = true;
+      ++g_armed;
       fence_async_smem();
-      mbar_expect_tx(bar_tma, 32768);
-      tma_load_3d(sG, &tm_g, 0, w % H_v, e.start, bar_tma);
+      mbar_arrive_expect_tx(bar_g, 32768);
+      tma_load_3d(sG, &tm_g, 0, w % H_v, e.start, bar_g);
     }
   };
   auto load_qk = [&](int w, const ChunkEntry &e, bool arrive) {
@@ -642,7 +652,10 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // the next item's, a whole item ahead of their use
     if (next < total) load_beta(next, ce_next, nbeta, ngsc);
   }
-  {
+  if constexpr (CHANNEL) {  // the gate tile; q, k, v are waited for after the decays
+    wait_bar(bar_g, it & 1, hdr, KDA_DEVICE_TIMEOUT);
+    if (!failed) g_done = it + 1;
+  } else {
     wait_bar(bar_tma, it & 1, hdr, KDA_DEVICE_TIMEOUT);
     if (!failed) tma_done = it + 1;
   }
@@ -725,6 +738,8 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   // the previous item's image copies must have read the X region before it is rebuilt
   if (tid == kIoThread) bulk_wait_read0();
   __syncthreads();  // g is consumed: the next item's lands there
+  wait_bar(bar_tma, it & 1, hdr, KDA_DEVICE_TIMEOUT);  // q, k, v
+  if (!failed) tma_done = it + 1;
   const bool exact = *s_exact != 0;  // CTA-uniform; reset after the operand pass
   if (tid == kIoThread && next < total && !exact) {
     load_g(next, ce_next);
@@ -1446,9 +1461,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
         mbar_arrive(bar_tma);
         ++tma_armed;
       }
-      // phases before tma_done were waited for at the top of their items
+      // phases before tma_done (g_done) were waited for in their items
       for (int ph = tma_done; ph < tma_armed; ++ph)
         mbar_wait(bar_tma, ph & 1, hdr, KDA_DEVICE_TIMEOUT);
+      for (int ph = g_done; ph < g_armed; ++ph)
+        mbar_wait(bar_g, ph & 1, hdr, KDA_DEVICE_TIMEOUT);
     }
     mbar_wait(bar_drain, 0, hdr, KDA_DEVICE_TIMEOUT);
   }
