@@ -18,9 +18,11 @@
  *
  * General conventions
  * -------------------
- *  - Every data pointer is a DEVICE pointer owned by the caller; the library
- *    allocates no device memory and keeps no state between calls except a
- *    per-device cache of attributes.  Work is enqueued on `stream` (a
+ *  - Every data pointer is a DEVICE pointer owned by the caller (except in
+ *    kda_chunk_fwd_host, which takes host memory).  The library allocates no
+ *    device memory (kda_chunk_fwd_noalloc's fixed array is part of its module)
+ *    and keeps no state between calls except a per-device cache of attributes
+ *    and kda_chunk_fwd_host's copy streams.  Work is enqueued on `stream` (a
  *    cudaStream_t; NULL = the legacy default stream) and the call returns
  *    without synchronising.
  *  - Token layout is [B, T, H, d] with d contiguous (equivalently [B*T, H, d]);
