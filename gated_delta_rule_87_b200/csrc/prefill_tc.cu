@@ -964,7 +964,9 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   //   a_t = e^{g_t}; e^{Gp_t} (K for W); e^{G_t} (q for Q');
   //   beta_t e^{G_L - G_t}, beta_t e^{G_L - Gp_t} (K_a, K_b);
   //   beta_t e^{E_J - G_t} (key column factor of the Gram blocks left of the diagonal).
-  // Rows past the chunk's length get 0 in the tile factors.
+  // Rows past the chunk's length get 0 in the tile factors.  (The exponentials
+  // use the intrinsic: its error is far below the bf16 rounding every factor
+  // meets in the operands.)
   float *tG = sPblk, *tGp = sPblk + 64, *tA = sPblk + 128, *tCW = sPblk + 192, *tE = sPblk + 256;
   float *tFK = sGsum, *tFQ = sGsum + 64, *tFA = sGsum + 128, *tFB = sGsum + 192;
   // diagonal-block factors [4 blocks][16 rows][kLdD] (the per-channel path's
@@ -985,20 +987,20 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     const float G0 = excl + g0, G1 = G0 + g1;
     const float GL = __shfl_sync(0xffffffffu, G1, 31);
     const float EJ = __shfl_sync(0xffffffffu, G1, lane | 7);  // end of this lane's 16-token block
-    const float gle = expf(GL);
+    const float gle = __expf(GL);
 #pragma unroll
     for (int h2 = 0; h2 < 2; ++h2) {
       const int t = t0 + h2;
-      const float Gt = h2 ? G1 : G0, Gpt = h2 ? G0 : excl, at = expf(h2 ? g1 : g0);
+      const float Gt = h2 ? G1 : G0, Gpt = h2 ? G0 : excl, at = __expf(h2 ? g1 : g0);
       const bool ok = t < L;
       const float b = sBeta[t];  // 0 past the chunk's length
-      const float fa = b * expf(GL - Gt);
+      const float fa = b * __expf(GL - Gt);
       tG[t] = Gt;
       tGp[t] = Gpt;
       tA[t] = at;
-      tCW[t] = b * expf(EJ - Gt);
-      tFK[t] = ok ? expf(Gpt) : 0.f;
-      tFQ[t] = ok ? expf(Gt) : 0.f;
+      tCW[t] = b * __expf(EJ - Gt);
+      tFK[t] = ok ? __expf(Gpt) : 0.f;
+      tFQ[t] = ok ? __expf(Gt) : 0.f;
       tFA[t] = fa;
       tFB[t] = fa * at;  // e^{G_L - Gp_t} = e^{G_L - G_t} e^{g_t}
       sGLe[t] = gle;
@@ -1011,7 +1013,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
     // of the decays a_s of tokens b < s < a (1 for b = a - 1, 0 for b >= a).
     // Products of factors <= 1: none overflows.
     const int I = (tid - 64) >> 4, a = (tid - 64) & 15;
-    const float own = expf(sGsc[16 * I + a]);  // a_{16I+a}
+    const float own = __expf(sGsc[16 * I + a]);  // a_{16I+a}
     float as[16];
 #pragma unroll
     for (int s2 = 0; s2 < 16; ++s2) as[s2] = __shfl_sync(0xffffffffu, own, (lane & 16) | s2);
@@ -1026,8 +1028,6 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
 #pragma unroll
     for (int q4 = 0; q4 < 4; ++q4) row[q4] = make_float4(d[4 * q4], d[4 * q4 + 1], d[4 * q4 + 2], d[4 * q4 + 3]);
   }
-  // the previous item's image copies must have read the X region before it is rebuilt
-  if (tid == kIoThread) bulk_wait_read0();
   __syncthreads();
   if (tid == kIoThread && next < total) {
     load_g(next, ce_next);
@@ -1068,6 +1068,11 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
   }
   __syncwarp();
   wait_bar(bar_mma, 0, hdr, KDA_DEVICE_TIMEOUT);
+  // The readback is the first to rebuild the X region (the tables and tiles
+  // above live elsewhere): only now must the previous item's image copies have
+  // read it, so their reads overlap this item's tables and image pass.
+  if (tid == kIoThread) bulk_wait_read0();
+  __syncthreads();
   tc_fence_after();
 
   // ---- 5'. Gram readback: TMEM lane r < 64 is key row i = r, lane 64 + t query
@@ -1099,7 +1104,7 @@ chunk_prep_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constan
       }
       const float rowg = isQ ? tG[r] : tGp[r];
       const bool rowok = r < L && J <= I;
-      const float rowf = (rowok && !diag) ? expf(rowg - tE[J]) : 0.f;
+      const float rowf = (rowok && !diag) ? __expf(rowg - tE[J]) : 0.f;
       tmem_ld_wait();
       if (diag) {
         // keys: beta_j D[a][u]; queries: beta_j D[a][u] a_t for u < a, beta_t at u = a
